@@ -1,0 +1,177 @@
+"""O0 oracle: scalar-loop brute force for tiny inputs -- TEST INFRASTRUCTURE ONLY.
+
+Plain Python floats (IEEE double) and explicit loops, written independently of
+``moe_oracle`` so that each pins the other.  Same sources and readings as
+``moe_oracle`` (GPT-OSS SwiGLU clip and alpha from "Ollama Imagegen GPT OSS",
+router/expert parameters from the MaxText GPT-OSS weight map, argsort
+dispatch and weighted combine from "Ollama glm4_moe_lite.go").
+
+Top-k here is found by enumerating every k-subset of experts, not by sorting;
+the dispatch permutation by counting, not by a library sort.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+import struct
+from typing import Dict, List, Sequence, Tuple
+
+
+def bf16_value(bits: int) -> float:
+    """Value of one bf16 bit pattern (the top half of an IEEE single)."""
+    return struct.unpack("<f", struct.pack("<I", (int(bits) & 0xFFFF) << 16))[0]
+
+
+def value(a) -> float:
+    """Scalar input value: numpy uint16 -> bf16, anything else -> float()."""
+    if getattr(a, "dtype", None) is not None and str(a.dtype) == "uint16":
+        return bf16_value(int(a))
+    return float(a)
+
+
+def e2m1(code: int) -> float:
+    """4-bit E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa."""
+    s = -1.0 if code & 8 else 1.0
+    e = (code >> 1) & 3
+    m = code & 1
+    if e == 0:
+        return s * (m / 2.0)
+    return s * (2.0 ** (e - 1)) * (1.0 + m / 2.0)
+
+
+def mxfp4_row(qrow, srow) -> List[float]:
+    """One dequantised weight row from packed bytes and E8M0 scale bytes."""
+    out = []
+    for i in range(len(qrow)):
+        byte = int(qrow[i])
+        for nib in (byte & 0xF, byte >> 4):
+            j = len(out)
+            out.append(e2m1(nib) * 2.0 ** (int(srow[j // 32]) - 127))
+    return out
+
+
+def weight_row(layer, name: str, e: int, n: int) -> List[float]:
+    w = layer[f"w_{name}"]
+    if str(w.dtype) == "uint8":
+        return mxfp4_row(w[e, n], layer[f"s_{name}"][e, n])
+    return [value(v) for v in w[e, n]]
+
+
+def sigmoid(z: float) -> float:
+    return 1.0 / (1.0 + math.exp(-z))
+
+
+def swiglu(g: float, u: float, limit: float, alpha: float = 1.702) -> float:
+    gc = g
+    if gc < 0.0:
+        gc = 0.0
+    if gc > limit:
+        gc = limit
+    uc = u
+    if uc < -limit:
+        uc = -limit
+    if uc > limit:
+        uc = limit
+    return gc * sigmoid(alpha * gc) * uc
+
+
+def dot(a: Sequence[float], b: Sequence[float]) -> float:
+    s = 0.0
+    for i in range(len(a)):
+        s += a[i] * b[i]
+    return s
+
+
+def router_logits(layer, t: int) -> List[float]:
+    x = [value(v) for v in layer["x"][t]]
+    E = layer["w_router"].shape[0]
+    return [dot(x, [value(v) for v in layer["w_router"][e]]) + value(layer["b_router"][e]) for e in range(E)]
+
+
+def topk_bruteforce(logits: Sequence[float], k: int) -> Tuple[List[int], List[float]]:
+    """The k-subset whose every member beats every non-member (ties: lower index wins).
+
+    Enumerates all subsets; returns the ids by descending logit and the softmax
+    over them.
+    """
+    E = len(logits)
+
+    def beats(a: int, b: int) -> bool:
+        return logits[a] > logits[b] or (logits[a] == logits[b] and a < b)
+
+    found = None
+    for sub in itertools.combinations(range(E), k):
+        rest = [e for e in range(E) if e not in sub]
+        if all(beats(a, b) for a in sub for b in rest):
+            found = list(sub)
+            break
+    assert found is not None
+    # order the chosen ids with a selection pass (no library sort)
+    ordered: List[int] = []
+    pool = list(found)
+    while pool:
+        best = pool[0]
+        for c in pool[1:]:
+            if beats(c, best):
+                best = c
+        ordered.append(best)
+        pool.remove(best)
+    m = max(logits[e] for e in ordered)
+    ex = [math.exp(logits[e] - m) for e in ordered]
+    z = sum(ex)
+    return ordered, [v / z for v in ex]
+
+
+def dispatch_counting(ids: Sequence[Sequence[int]], E: int) -> Tuple[List[int], List[List[int]], List[int]]:
+    """Counting-sort dispatch: segment offsets, row of each (t, j), slot of each row."""
+    T = len(ids)
+    k = len(ids[0]) if T else 0
+    cnt = [0] * E
+    for t in range(T):
+        for j in range(k):
+            cnt[ids[t][j]] += 1
+    off = [0] * (E + 1)
+    for e in range(E):
+        off[e + 1] = off[e] + cnt[e]
+    fill = list(off[:E])
+    row_of_slot = [[-1] * k for _ in range(T)]
+    slot_of_row = [-1] * (T * k)
+    for t in range(T):            # increasing token order -> stable by token
+        for j in range(k):
+            e = ids[t][j]
+            r = fill[e]
+            fill[e] += 1
+            row_of_slot[t][j] = r
+            slot_of_row[r] = t * k + j
+    return off, row_of_slot, slot_of_row
+
+
+def expert_output(layer, e: int, x: Sequence[float], limit: float, alpha: float = 1.702) -> Tuple[List[float], List[float]]:
+    """(h, o) of expert e for one activation row, by scalar loops."""
+    F = layer["b_gate"].shape[1]
+    D = layer["b_down"].shape[1]
+    h = []
+    for f in range(F):
+        g = dot(x, weight_row(layer, "gate", e, f)) + value(layer["b_gate"][e, f])
+        u = dot(x, weight_row(layer, "up", e, f)) + value(layer["b_up"][e, f])
+        h.append(swiglu(g, u, limit, alpha))
+    o = []
+    for d in range(D):
+        o.append(dot(h, weight_row(layer, "down", e, d)) + value(layer["b_down"][e, d]))
+    return h, o
+
+
+def layer_token(layer, t: int, k: int, limit: float, alpha: float = 1.702) -> Dict[str, list]:
+    """The whole layer for token t, by scalar loops."""
+    lg = router_logits(layer, t)
+    ids, w = topk_bruteforce(lg, k)
+    x = [value(v) for v in layer["x"][t]]
+    D = layer["b_down"].shape[1]
+    y = [0.0] * D
+    hs = []
+    for j in range(k):
+        h, o = expert_output(layer, ids[j], x, limit, alpha)
+        hs.append(h)
+        for d in range(D):
+            y[d] += w[j] * o[d]
+    return dict(logits=lg, ids=ids, w=w, h=hs, y=y)
