@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Benchmark of the GPT-OSS MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one whole layer forward (router + top-k, dispatch, gate/up GEMM +
+clipped SwiGLU, down GEMM + weighted un-permutation, combine) over one batch
+of T synthetic tokens already resident in HBM, through the C ABI call
+moe_layer_forward.  Default workload: the GPT-OSS-20B-shaped prefill layer
+(T=4096, D=F=2880, E=32, k=4, bf16).  Inputs and weights are seeded synthetic
+tensors (random-init weights of that shape); the expert weights (1.6 GB) are
+far larger than L2, so consecutive steps cannot be served from L2.
+
+Under torchrun (N > 1) every rank runs an independent replica on its own
+tokens (data parallel, weak scaling, no collective on the data path); the
+step time is the max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (numpy fp64, the plain definition of
+the layer) on this host's cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "MoE layer tokens/s + TFLOP/s vs TC peak (prefill); GB/s vs HBM peak (decode)"
+STAGES = ("router_topk", "dispatch", "gateup_swiglu_gemm", "down_combine_gemm", "combine")
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", default="gptoss20b_prefill", choices=sorted(W.SPECS))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(bf16_tflops=d["bf16_tflops"], bf16_tflops_sustained=d["bf16_tflops_sustained"],
+                    hbm_gbs=d["hbm_gbs"], source="measured")
+    return dict(bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, hbm_gbs=6650.0, source="fallback")
+
+
+def config_of(spec, n_gpus):
+    return {"workload": spec.name, "T_per_gpu": spec.T, "hidden_size": spec.D, "intermediate_size": spec.F,
+            "num_local_experts": spec.E, "num_experts_per_tok": spec.k, "swiglu_limit": spec.limit,
+            "expert_weights": spec.wfmt, "global_tokens": spec.T * n_gpus,
+            "parallelism": f"dp{n_gpus} (independent replicas)",
+            "l2": "inputs larger than L2: every step streams all expert weights "
+                  f"({expert_weight_bytes(spec) / 1e9:.2f} GB) through HBM"}
+
+
+def expert_weight_bytes(spec):
+    n = 3 * spec.E * spec.D * spec.F
+    return n * (2 if spec.dtype == "bf16" else 4) if spec.wfmt == "dense" else n // 2 + n // 32
+
+
+# --------------------------------------------------------------------------- #
+# clocks during the timed region (NVML reads only)
+# --------------------------------------------------------------------------- #
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.err = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:   # no NVML: report that instead of clocks
+            self.nv, self.err, self.max_mhz = None, repr(e), None
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name not in ("gpu_idle",):
+                        self.reasons.add(name)
+            except Exception as e:
+                self.err = repr(e)
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv is not None:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0, "error": self.err}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- #
+# CPU oracle timing (the reference arm and the cpu_baseline leg)
+# --------------------------------------------------------------------------- #
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_step(spec, layer, S):
+    """The oracle (as it stands) on the first S tokens of the workload: whole layer, every expert decoded."""
+    from oracle import moe_oracle as O
+    sub = dict(layer)
+    sub["x"] = layer["x"][:S]
+    t0 = time.perf_counter()
+    O.layer_forward(sub, spec.k, spec.limit, spec.alpha)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(spec, layer, budget_s=20.0):
+    S = 32
+    dt = oracle_step(spec, layer, S)
+    while dt < budget_s / 4 and S < spec.T:
+        S = min(spec.T, S * 4)
+        dt = oracle_step(spec, layer, S)
+    return {"value": S / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {S} of {spec.T} tokens through the whole layer (numpy fp64, all "
+                      f"{spec.E} experts decoded), {dt:.1f} s"}
+
+
+def oracle_tokens_step(spec, layer, S):
+    """The oracle (as it stands) for the first S tokens, one token at a time (only their experts decoded)."""
+    from oracle import moe_oracle as O
+    t0 = time.perf_counter()
+    O.layer_tokens(layer, np.arange(S), spec.k, spec.limit, spec.alpha)
+    return time.perf_counter() - t0
+
+
+def run_reference(args, rank, world, budget_s=150.0):
+    if rank != 0:
+        return
+    spec = W.SPECS[args.workload]
+    layer = W.make_layer(spec, seed=0)
+    # size the per-step sample so that warm-up + timed steps fit in about budget_s
+    per_step = budget_s / max(1, args.steps + args.warmup)
+    S = 1
+    dt = oracle_tokens_step(spec, layer, S)
+    while S < spec.T and dt * 2.5 < per_step:
+        S = min(spec.T, S * 2)
+        dt = oracle_tokens_step(spec, layer, S)
+    for _ in range(args.warmup):
+        oracle_tokens_step(spec, layer, S)
+    t = [oracle_tokens_step(spec, layer, S) for _ in range(args.steps)]
+    ms = 1e3 * sum(t) / len(t)
+    value = S / (ms / 1e3)
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_of(spec, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"each step: the first {S} of {spec.T} tokens, each through the "
+                                       "router and its k experts (numpy fp64; the chosen experts' weights "
+                                       "decoded once per step)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "impl": "reference"}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- #
+# our arm
+# --------------------------------------------------------------------------- #
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_ffn_12_b200 import _lib, api
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    spec = W.SPECS[args.workload]
+    layer = W.make_layer(spec, seed=0)
+    if rank > 0:   # each replica routes its own tokens
+        layer["x"] = W.make_layer(spec, seed=rank, with_experts=False)["x"]
+    d = api.upload_layer(layer, dev)
+    cfg = api.config_from_spec(spec)
+    moe = api.MoELayer(cfg, d["w_router"], d["b_router"], api.expert_weights_from(d))
+    x, T = d["x"], spec.T
+    y = torch.empty_like(x)
+    moe.workspace(T)
+    lib = _lib.load()
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        return reduce_max(v, dev)
+
+    for _ in range(max(args.warmup, 3)):
+        moe(x, y=y)
+    torch.cuda.synchronize()
+    if api.last_device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    # per-step stage events, recorded by the library on this stream
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(STAGES))] for _ in range(K)]
+    for row in ev:
+        for e in row:
+            e.record(stream)   # materialise the handles
+    torch.cuda.synchronize()
+    handles = [[ctypes_ptr(e.cuda_event) for e in row] for row in ev]
+    n = len(STAGES)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    sampler = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        launches0 = lib.moe_launch_count()
+        t0.record(stream)
+        for i in range(K):
+            starts = (_lib.ctypes.c_void_p * n)(*handles[i][:n])
+            stops = (_lib.ctypes.c_void_p * n)(*handles[i][n:])
+            lib.moe_set_stage_events(starts, stops, n)
+            moe(x, y=y)
+        t1.record(stream)
+        lib.moe_set_stage_events(None, None, 0)
+        launches = lib.moe_launch_count() - launches0
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    if api.last_device_error() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    stage_ms = {name: statistics.mean(ev[i][s].elapsed_time(ev[i][n + s]) for i in range(K))
+                for s, name in enumerate(STAGES)}
+
+    # end to end: pinned host input -> device, layer, device -> pinned host output, every step
+    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    x_host.copy_(x)
+    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    x_dev = torch.empty_like(x)
+    for _ in range(3):
+        x_dev.copy_(x_host, non_blocking=True)
+        moe(x_dev, y=y)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    Ke = max(5, K // 4)
+    e0.record(stream)
+    for _ in range(Ke):
+        x_dev.copy_(x_host, non_blocking=True)
+        moe(x_dev, y=y)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(spec, layer)
+
+    if rank == 0:
+        peaks = measured_peaks()
+        flops = spec.expert_flops() + spec.router_flops()
+        ms_step = ms_total / K
+        value = job_throughput(world, T, K, ms_total)
+        gu_flops = 4.0 * spec.R * spec.D * spec.F
+        gu_ms = stage_ms["gateup_swiglu_gemm"]
+        achieved = gu_flops / (gu_ms / 1e3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if spec.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded random-init weights and activations of the GPT-OSS-20B MoE layer shape)",
+            "config": config_of(spec, world),
+            "tflops": flops / (ms_step / 1e3) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": "gateup_swiglu_gemm", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "peak_source": peaks["source"] + " bf16 burst",
+                         "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                         "flops_per_launch": gu_flops, "ms_per_launch": gu_ms,
+                         "traffic": traffic_from_profiles("gateup_swiglu_gemm", spec.name)},
+            "stage_ms": stage_ms,
+            "layer_tflops_frac": flops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "e2e": {"value": job_throughput(world, T, Ke, ms_e2e), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+            "gpu_launches": int(launches),
+            "clocks": sampler.summary(),
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def reduce_max(v: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank processed tokens_per_rank tokens per step; time = slowest rank."""
+    return world * tokens_per_rank * steps / (ms_max / 1e3)
+
+
+def ctypes_ptr(h):
+    from mixture_experts_ffn_12_b200 import _lib
+    return _lib.ctypes.c_void_p(int(h)).value
+
+
+def traffic_from_profiles(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    src = os.path.join(ROOT, "mixture_experts_ffn_12_b200", "csrc", "grouped_gemm.cuh")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(path):
+        if ":" in line and line.startswith("- "):
+            k, v = line[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != sha:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,206 @@
+/*
+ * moe.h -- C ABI of libmoe: the GPT-OSS Mixture-of-Experts FFN layer on B200 (sm_100a).
+ *
+ * The layer (per token t, with D = hidden_size, E = num_local_experts,
+ * k = num_experts_per_tok, F = intermediate_size, L = swiglu_limit):
+ *   l[t,e]  = x[t] . Wr[e] + br[e]                      router kernel + bias
+ *             (MaxText GPT-OSS weight map, "MoE Router")
+ *   S_t     = the k largest l[t,.], descending, ties -> lower expert index
+ *   w[t,j]  = softmax over {l[t,e] : e in S_t}
+ *   for e in S_t:
+ *     g = x[t] Wg[e]^T + bg[e],  u = x[t] Wu[e]^T + bu[e]   (wi_0 / wi_1 with biases,
+ *                                                         MaxText "MOE EXPERTS")
+ *     h = clip(g,0,L) * sigmoid(alpha clip(g,0,L)) * clip(u,-L,L), alpha = 1.702
+ *         ("Ollama Imagegen GPT OSS", Description: the clipped SwiGLU)
+ *     o_e = h Wd[e]^T + bd[e]                            (wo with bias)
+ *   y[t]    = sum_j w[t,j] o_{S_t[j]}                    ("Ollama glm4_moe_lite.go", MoE.Forward)
+ * The config mirrors the GPT-OSS Config struct (hidden_size, num_local_experts,
+ * num_experts_per_tok, swiglu_limit; "Ollama Imagegen GPT OSS", Signature).
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *    16-byte aligned.  The library never allocates or frees device memory and
+ *    never synchronises the host on these calls; work is enqueued on `stream`
+ *    (a cudaStream_t, NULL = the legacy default stream) of the current device.
+ *  - Weights are stored K-major ("[N, K]", the reduction dim contiguous):
+ *      w_router [E, D]; w_gate, w_up [E, F, D]; w_down [E, D, F];
+ *      b_router [E]; b_gate, b_up [E, F]; b_down [E, D].
+ *    Activations, router and dense expert weights, biases and outputs use
+ *    `dtype` (fp32 or bf16).  Routing weights are always fp32, ids int32.
+ *  - MXFP4 expert weights (wfmt = MOE_W_MXFP4, dtype must be bf16): packed
+ *    E2M1 codes [.., N, K/2] uint8 (element 2i = low nibble of byte i, code bit 3
+ *    = sign, bits 2..1 = exponent with bias 1, bit 0 = mantissa) and E8M0 scale
+ *    bytes [.., N, K/32] (scale 2^(s-127) for 32 consecutive elements along K),
+ *    per the OCP Microscaling formats; the pages name the format "MXFP4"
+ *    ("GPT-OSS 20B GGUF with MoE CPU Offloading", Model Specifications).
+ *  - Arguments are validated before any launch; a rejected call launches
+ *    nothing and returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED /
+ *    MOE_ERR_WORKSPACE.  T = 0 is a successful no-op (expert_off is zeroed
+ *    where it is an output).  Launch failures return MOE_ERR_CUDA.
+ *  - Faults found on the device (an out-of-range id or row index read from a
+ *    caller buffer, a bounded wait that gave up) never trap: the kernels skip
+ *    the access or end early and set a per-device error word, which
+ *    moe_last_device_error() reads after a synchronisation.  Results of such a
+ *    call are unspecified.
+ *  - Supported sizes: 1 <= k <= min(E, 8), 1 <= E <= 256, D and F multiples of
+ *    16 (of 32 for MXFP4), T >= 0 with T*k < 2^31; swiglu_limit finite and > 0.
+ *  - NaN/Inf inputs: unspecified.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or config field */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but not supported (e.g. MXFP4 with fp32 activations) */
+  MOE_ERR_WORKSPACE = 3,    /* workspace pointer null or smaller than the size function says */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  MOE_ERR_TIMEOUT = 5,      /* moe_last_device_error: a kernel's bounded wait gave up */
+  MOE_ERR_DEVICE_BOUNDS = 6 /* moe_last_device_error: an index read on the device was out of range */
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+typedef enum { MOE_W_DENSE = 0, MOE_W_MXFP4 = 1 } moe_wfmt_t;
+
+/* Field names follow the GPT-OSS Config (hidden_size, num_local_experts,
+ * num_experts_per_tok, swiglu_limit); intermediate_size is F. */
+typedef struct {
+  int32_t hidden_size;         /* D */
+  int32_t intermediate_size;   /* F */
+  int32_t num_local_experts;   /* E */
+  int32_t num_experts_per_tok; /* k */
+  float swiglu_limit;          /* L, e.g. 7.0 */
+  float swiglu_alpha;          /* 1.702 for GPT-OSS */
+  int32_t dtype;               /* moe_dtype_t */
+  int32_t wfmt;                /* moe_wfmt_t */
+} moe_config_t;
+
+/* Expert parameters (device pointers).  Dense: w_* in dtype, s_* NULL.
+ * MXFP4: w_* packed E2M1 uint8, s_* E8M0 uint8.  Biases always in dtype. */
+typedef struct {
+  const void* w_gate;     /* [E, F, D]   (MXFP4: [E, F, D/2]) */
+  const void* w_up;       /* [E, F, D]   (MXFP4: [E, F, D/2]) */
+  const void* w_down;     /* [E, D, F]   (MXFP4: [E, D, F/2]) */
+  const uint8_t* s_gate;  /* MXFP4: [E, F, D/32] */
+  const uint8_t* s_up;    /* MXFP4: [E, F, D/32] */
+  const uint8_t* s_down;  /* MXFP4: [E, D, F/32] */
+  const void* b_gate;     /* [E, F] */
+  const void* b_up;       /* [E, F] */
+  const void* b_down;     /* [E, D] */
+} moe_expert_weights_t;
+
+/* ABI version of the loaded library (MOE_ABI_VERSION). */
+MOE_API int32_t moe_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+MOE_API const char* moe_status_string(moe_status_t status);
+
+/* Checks a config without touching the GPU: MOE_OK or the reason it is rejected. */
+MOE_API moe_status_t moe_config_check(const moe_config_t* cfg);
+
+/* Bytes of workspace moe_permute needs for T tokens (its histogram and scan
+ * scratch).  0 when T == 0; (size_t)-1 if cfg is invalid. */
+MOE_API size_t moe_permute_workspace_size(const moe_config_t* cfg, int64_t T);
+
+/* Bytes of workspace moe_expert_ffn needs (0 for dense weights; MXFP4 needs room
+ * for dequantised expert weights). (size_t)-1 if cfg is invalid. */
+MOE_API size_t moe_expert_ffn_workspace_size(const moe_config_t* cfg, int64_t T);
+
+/* Bytes of workspace moe_layer_forward needs for T tokens: routing ids and
+ * weights, dispatch maps, permuted activations x_perm [T*k, D], the SwiGLU
+ * output h [T*k, F], the weighted expert outputs [T*k, D] in fp32 (sharing
+ * x_perm's space), plus what the sub-steps need.  (size_t)-1 if cfg is invalid. */
+MOE_API size_t moe_workspace_size(const moe_config_t* cfg, int64_t T);
+
+/* Router + top-k + softmax (steps l, S_t, w above).
+ *   x [T, D], w_router [E, D], b_router [E] in dtype
+ *   -> topk_ids [T, k] int32 (descending logit, ties -> lower index),
+ *      topk_w   [T, k] fp32 (softmax over the k selected logits).
+ * The logits are accumulated in fp32 (bf16 products are exact in fp32; fp32
+ * inputs use fp32 FMA, never TF32). */
+MOE_API moe_status_t moe_router_topk(const moe_config_t* cfg, int64_t T, const void* x, const void* w_router,
+                             const void* b_router, int32_t* topk_ids, float* topk_w, void* stream);
+
+/* Dispatch: the stable sort of the T*k (token, slot) pairs by expert id
+ * ("Ollama glm4_moe_lite.go", SwitchMLP.Forward: argsort of the flattened ids).
+ *   topk_ids [T, k] int32 (distinct per token, each in [0, E)),
+ *   x [T, D] dtype (may be NULL together with x_perm: index maps only)
+ *   -> expert_off  [E+1] int32: rows of expert e are [expert_off[e], expert_off[e+1]),
+ *      row_of_slot [T*k] int32: permuted row of pair (t, j) at index t*k+j,
+ *      slot_of_row [T*k] int32: t*k+j of the pair held by each permuted row,
+ *      x_perm [T*k, D] dtype:   x_perm[r] = x[slot_of_row[r] / k].
+ * Rows of one expert are in increasing token order.  Deterministic.
+ * ws: moe_permute_workspace_size(cfg, T) bytes of device scratch. */
+MOE_API moe_status_t moe_permute(const moe_config_t* cfg, int64_t T, const int32_t* topk_ids, const void* x,
+                         int32_t* expert_off, int32_t* row_of_slot, int32_t* slot_of_row, void* x_perm, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* Per-expert FFN over the permuted rows (R = T*k):
+ *   x_perm [R, D], expert_off [E+1] (as produced by moe_permute; read on the device)
+ *   -> h [R, F]: clipped SwiGLU of the gate/up projections (+ biases),
+ *      y_perm [R, D]: h Wd[e]^T + bd[e] for the expert e that owns each row.
+ * Computed on the tcgen05 tensor cores with fp32 accumulation (bf16 operands;
+ * fp32 layers use TF32 operands).  ws: moe_expert_ffn_workspace_size bytes
+ * (may be NULL when that is 0). */
+MOE_API moe_status_t moe_expert_ffn(const moe_config_t* cfg, int64_t T, const void* x_perm, const int32_t* expert_off,
+                            const moe_expert_weights_t* weights, void* h, void* y_perm, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* Weighted combine: y[t] = sum_{j<k} topk_w[t,j] * y_perm[row_of_slot[t,j]],
+ * summed in fp32 in fixed j order.  y_perm [T*k, D], y [T, D] in dtype. */
+MOE_API moe_status_t moe_combine(const moe_config_t* cfg, int64_t T, const void* y_perm, const int32_t* row_of_slot,
+                         const float* topk_w, void* y, void* stream);
+
+/* The whole layer: router/top-k -> dispatch -> gate/up + SwiGLU -> down with
+ * the routing weight and the un-permutation fused into its epilogue -> sum
+ * over k.  x [T, D], y [T, D] in dtype.  topk_ids_out [T, k] and topk_w_out
+ * [T, k] are optional (NULL: kept in the workspace).  ws: moe_workspace_size
+ * bytes. */
+MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x, const void* w_router,
+                               const void* b_router, const moe_expert_weights_t* weights, void* y,
+                               int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Reads and clears the current device's error word (synchronises the device).
+ * MOE_OK if no kernel flagged anything since the last call, MOE_ERR_TIMEOUT if a
+ * bounded wait gave up, MOE_ERR_DEVICE_BOUNDS if an index read on the device was
+ * out of range, MOE_ERR_CUDA if the read itself failed. */
+MOE_API moe_status_t moe_last_device_error(void);
+
+/* Profiling aid: CUDA events recorded around the stages of moe_layer_forward
+ * (and the gate/up and down stages of moe_expert_ffn).  starts[i] and
+ * stops[i] (cudaEvent_t handles, may be NULL) are recorded on the call's
+ * stream right before and right after stage i: 0 router + top-k, 1 dispatch,
+ * 2 gate/up GEMM + SwiGLU, 3 down GEMM (+ weighting and un-permutation),
+ * 4 combine.  n <= 5 entries are copied; they apply to every later call in
+ * this process until the next call of this function (n = 0 clears). */
+MOE_API void moe_set_stage_events(void* const* starts, void* const* stops, int32_t n);
+
+/* Number of kernels this library has launched in this process so far. */
+MOE_API uint64_t moe_launch_count(void);
+
+/* Time limit, in nanoseconds, of every bounded wait inside the kernels
+ * launched afterwards by this process (default 1e9 = 1 s; 0 restores the
+ * default).  A debugging aid: a tiny limit makes waits give up early, which
+ * moe_last_device_error then reports. */
+MOE_API void moe_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

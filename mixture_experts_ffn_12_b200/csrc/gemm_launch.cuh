@@ -1,0 +1,203 @@
+#pragma once
+// Host side of the tcgen05 grouped GEMMs: TMA tensor maps and launches.
+//
+//   router (bf16, many tokens)  A = x [T, D],        B = Wr [1, E, D],   EPI_TOPK
+//   gate/up                     A = x_perm [R, D],   B = W_g, W_u [E, F, D], EPI_SWIGLU
+//   down                        A = h [R, F],        B = W_d [E, D, F],  EPI_BIAS / EPI_BIAS_WSCATTER
+//
+// fp32 layers use the fp32-FMA grouped GEMM of simt_gemm.cuh instead.
+// Every operand is K-major; tensor maps cut [rows x 128 B] boxes with the
+// 128-byte swizzle, out-of-range rows and columns read as zero (ragged expert
+// segments, the last column block of F or D, a partial last K block).
+#include <mutex>
+
+#include "grouped_gemm.cuh"
+#include "internal.h"
+#include "simt_gemm.cuh"
+
+namespace moe {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// K-major matrix: [rows, K] (groups == 0) or [groups, rows, K]; box = box_rows x 128 bytes.
+static cudaError_t make_tmap(CUtensorMap* m, const void* ptr, bool f32, uint64_t K, uint64_t rows, uint64_t groups,
+                             uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const uint64_t elem = f32 ? 4 : 2;
+  const cuuint64_t dims[3] = {K, rows, groups ? groups : 1};
+  const cuuint64_t strides[2] = {K * elem, K * elem * rows};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kRowBytes / elem), box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        groups ? 3 : 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <typename T, int TN, int NB, int EPI, int STAGES>
+static cudaError_t launch(const Launch& L, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                          const GemmArgs& args, int64_t max_tiles) {
+  if (max_tiles <= 0) return cudaSuccess;
+  auto kern = grouped_gemm_kernel<T, TN, NB, EPI, STAGES>;
+  constexpr int smem = GemmLayout<TN, NB>::smem_bytes(STAGES);
+  static_assert(smem <= 232448, "shared memory budget");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static std::mutex mu;
+  static uint64_t configured = 0;   // one bit per device
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (dev >= 64 || !((configured >> dev) & 1u)) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) configured |= uint64_t(1) << dev;
+    }
+  }
+  const int grid = static_cast<int>(std::min<int64_t>(max_tiles, L.num_sms));
+  kern<<<grid, kGemmThreads, smem, L.stream>>>(a, b0, b1, args);
+  count_launch();
+  return cudaGetLastError();
+}
+
+static GemmArgs base_args(const Launch& L) {
+  GemmArgs a{};
+  a.wait_limit_ns = L.wait_limit_ns;
+  a.alpha = 1.702f;
+  return a;
+}
+
+static int64_t max_row_blocks(int64_t R, int G) { return (R + kBM - 1) / kBM + G; }
+
+constexpr int kStages = 4;
+constexpr int kTNGateUp = 120;   // 2 x 120 = 240 MMA columns, F = 2880 = 24 x 120
+constexpr int kTNDown = 240;     // D = 2880 = 12 x 240
+
+cudaError_t router_tc(const Launch& L, int64_t T, int D, int E, int k, const void* x, const void* w_router,
+                      const void* b_router, int32_t* ids, float* w) {
+  const int mma_n = (E + 15) / 16 * 16;
+  CUtensorMap ta, tb;
+  cudaError_t e;
+  if ((e = make_tmap(&ta, x, false, D, T, 0, kBM)) != cudaSuccess) return e;
+  if ((e = make_tmap(&tb, w_router, false, D, E, 1, mma_n)) != cudaSuccess) return e;
+  GemmArgs a = base_args(L);
+  a.group_off = nullptr;
+  a.num_groups = 1;
+  a.m_total = static_cast<int>(T);
+  a.n_out = E;
+  a.k_dim = D;
+  a.mma_n = mma_n;
+  a.bias0 = b_router;
+  a.topk_ids = ids;
+  a.topk_wout = w;
+  a.topk_k = k;
+  return launch<__nv_bfloat16, 256, 1, EPI_TOPK, kStages>(L, ta, tb, tb, a, (T + kBM - 1) / kBM);
+}
+
+cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,
+                          const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h) {
+  if (R == 0) return cudaSuccess;
+  if (!bf16) {
+    GemmArgs a = base_args(L);
+    a.group_off = expert_off;
+    a.num_groups = E;
+    a.m_total = static_cast<int>(R);
+    a.n_out = F;
+    a.k_dim = D;
+    a.bias0 = w.b_gate;
+    a.bias1 = w.b_up;
+    a.limit = limit;
+    a.alpha = alpha;
+    a.out = h;
+    a.ldo = F;
+    const dim3 grid((F + kSimtBN - 1) / kSimtBN, static_cast<unsigned>((R + kSimtBM - 1) / kSimtBM + E));
+    simt_grouped_gemm_f32<EPI_SWIGLU><<<grid, 256, 0, L.stream>>>(
+        static_cast<const float*>(x_perm), static_cast<const float*>(w.w_gate), static_cast<const float*>(w.w_up), a);
+    count_launch();
+    return cudaGetLastError();
+  }
+  CUtensorMap ta, tg, tu;
+  cudaError_t e;
+  if ((e = make_tmap(&ta, x_perm, !bf16, D, R, 0, kBM)) != cudaSuccess) return e;
+  if ((e = make_tmap(&tg, w.w_gate, !bf16, D, F, E, kTNGateUp)) != cudaSuccess) return e;
+  if ((e = make_tmap(&tu, w.w_up, !bf16, D, F, E, kTNGateUp)) != cudaSuccess) return e;
+  GemmArgs a = base_args(L);
+  a.group_off = expert_off;
+  a.num_groups = E;
+  a.m_total = static_cast<int>(R);
+  a.n_out = F;
+  a.k_dim = D;
+  a.bias0 = w.b_gate;
+  a.bias1 = w.b_up;
+  a.limit = limit;
+  a.alpha = alpha;
+  a.out = h;
+  a.ldo = F;
+  const int64_t tiles = max_row_blocks(R, E) * ((F + kTNGateUp - 1) / kTNGateUp);
+  return launch<__nv_bfloat16, kTNGateUp, 2, EPI_SWIGLU, kStages>(L, ta, tg, tu, a, tiles);
+}
+
+cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* h,
+                        const int32_t* expert_off, const ExpertWeights& w, const int32_t* slot_of_row,
+                        const float* topk_w, void* out) {
+  if (R == 0) return cudaSuccess;
+  if (!bf16) {
+    GemmArgs a = base_args(L);
+    a.group_off = expert_off;
+    a.num_groups = E;
+    a.m_total = static_cast<int>(R);
+    a.n_out = D;
+    a.k_dim = F;
+    a.bias0 = w.b_down;
+    a.out = out;
+    a.ldo = D;
+    a.slot_of_row = slot_of_row;
+    a.topk_w = topk_w;
+    const dim3 grid((D + kSimtBN - 1) / kSimtBN, static_cast<unsigned>((R + kSimtBM - 1) / kSimtBM + E));
+    if (slot_of_row != nullptr)
+      simt_grouped_gemm_f32<EPI_BIAS_WSCATTER><<<grid, 256, 0, L.stream>>>(
+          static_cast<const float*>(h), static_cast<const float*>(w.w_down), nullptr, a);
+    else
+      simt_grouped_gemm_f32<EPI_BIAS><<<grid, 256, 0, L.stream>>>(static_cast<const float*>(h),
+                                                                  static_cast<const float*>(w.w_down), nullptr, a);
+    count_launch();
+    return cudaGetLastError();
+  }
+  CUtensorMap ta, tb;
+  cudaError_t e;
+  if ((e = make_tmap(&ta, h, !bf16, F, R, 0, kBM)) != cudaSuccess) return e;
+  if ((e = make_tmap(&tb, w.w_down, !bf16, F, D, E, kTNDown)) != cudaSuccess) return e;
+  GemmArgs a = base_args(L);
+  a.group_off = expert_off;
+  a.num_groups = E;
+  a.m_total = static_cast<int>(R);
+  a.n_out = D;
+  a.k_dim = F;
+  a.bias0 = w.b_down;
+  a.out = out;
+  a.ldo = D;
+  a.slot_of_row = slot_of_row;
+  a.topk_w = topk_w;
+  const int64_t tiles = max_row_blocks(R, E) * ((D + kTNDown - 1) / kTNDown);
+  if (slot_of_row != nullptr)
+    return launch<__nv_bfloat16, kTNDown, 1, EPI_BIAS_WSCATTER, kStages>(L, ta, tb, tb, a, tiles);
+  return launch<__nv_bfloat16, kTNDown, 1, EPI_BIAS, kStages>(L, ta, tb, tb, a, tiles);
+}
+
+}  // namespace moe

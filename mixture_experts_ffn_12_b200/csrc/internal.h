@@ -1,0 +1,63 @@
+// Host-side internal interface between the C ABI (moe_abi.cu) and the kernel
+// launchers.  Not installed; the public interface is include/moe.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <atomic>
+
+namespace moe {
+
+// Kernels this library has launched in this process (moe_launch_count).
+inline std::atomic<uint64_t> g_launches{0};
+inline void count_launch(uint64_t n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+struct Launch {
+  cudaStream_t stream;
+  int num_sms;
+  unsigned long long wait_limit_ns;
+};
+
+// Router + top-k + softmax.  ids/w are [T, k].
+cudaError_t router_topk(const Launch& L, bool bf16, int64_t T, int D, int E, int k, const void* x,
+                        const void* w_router, const void* b_router, int32_t* ids, float* w);
+
+// Scratch (int32 words) the permute needs for T tokens and E experts.
+size_t permute_scratch_words(int64_t T, int E);
+
+// Dispatch: expert_off [E+1], row_of_slot [T*k], slot_of_row [T*k], x_perm [T*k, D].
+// x / x_perm may be null (index maps only).
+cudaError_t permute(const Launch& L, bool bf16, int64_t T, int D, int E, int k, const int32_t* ids,
+                    const void* x, int32_t* expert_off, int32_t* row_of_slot, int32_t* slot_of_row,
+                    void* x_perm, int32_t* scratch);
+
+struct ExpertWeights {
+  const void *w_gate, *w_up, *w_down;        // dense [E,F,D],[E,F,D],[E,D,F]; MXFP4: packed [..,K/2]
+  const uint8_t *s_gate, *s_up, *s_down;     // MXFP4 scales [..,K/32]
+  const void *b_gate, *b_up, *b_down;        // [E,F],[E,F],[E,D]
+};
+
+// h[R, F] = swiglu(x_perm W_g^T + b_g, x_perm W_u^T + b_u), per expert segment.
+cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,
+                          const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h);
+
+// Down projection.  If slot_of_row == nullptr: out[r] = h[r] W_d^T + b_d (permuted order, dtype);
+// else out[slot_of_row[r]] = topk_w[slot] * (h[r] W_d^T + b_d) (slot order, fp32).
+cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* h,
+                        const int32_t* expert_off, const ExpertWeights& w, const int32_t* slot_of_row,
+                        const float* topk_w, void* out);
+
+// y[t] = sum_j w[t,j] * y_perm[row_of_slot[t,j]]
+cudaError_t combine_gather(const Launch& L, bool bf16, int64_t T, int D, int k, const void* y_perm,
+                           const int32_t* row_of_slot, const float* w, void* y);
+// y[t] = sum_j ys[t*k + j]   (ys fp32, y dtype)
+cudaError_t combine_slots(const Launch& L, bool bf16, int64_t T, int D, int k, const void* ys, void* y);
+
+// MXFP4 -> bf16 weights ([rows, K/2] packed + [rows, K/32] scales -> [rows, K]).
+cudaError_t mxfp4_dequant(const Launch& L, int64_t rows, int K, const uint8_t* q, const uint8_t* s, void* out);
+
+cudaError_t read_and_clear_device_error(int* bits);
+
+}  // namespace moe

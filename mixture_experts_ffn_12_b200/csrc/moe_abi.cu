@@ -1,0 +1,344 @@
+// extern "C" entry points of libmoe (declared and documented in include/moe.h):
+// argument validation, workspace carving, and the sequence of launches.
+// The library is built from this single translation unit.
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "internal.h"
+// one translation unit: the kernels share the per-device error word
+#include "router_permute_combine.cuh"
+#include "gemm_launch.cuh"
+
+namespace {
+
+using moe::Launch;
+
+std::atomic<unsigned long long> g_wait_limit_ns{1000000000ull};
+
+// stage events (moe_set_stage_events)
+constexpr int kStages = 5;
+enum { ST_ROUTER = 0, ST_DISPATCH = 1, ST_GATEUP = 2, ST_DOWN = 3, ST_COMBINE = 4 };
+std::mutex g_ev_mu;
+cudaEvent_t g_ev_start[kStages] = {};
+cudaEvent_t g_ev_stop[kStages] = {};
+
+void stage_mark(int stage, bool start, cudaStream_t st) {
+  cudaEvent_t ev;
+  {
+    std::lock_guard<std::mutex> g(g_ev_mu);
+    ev = start ? g_ev_start[stage] : g_ev_stop[stage];
+  }
+  if (ev != nullptr) cudaEventRecord(ev, st);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+moe_status_t check_cfg(const moe_config_t* c) {
+  if (c == nullptr) return MOE_ERR_INVALID_ARG;
+  const int D = c->hidden_size, F = c->intermediate_size, E = c->num_local_experts, k = c->num_experts_per_tok;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->wfmt != MOE_W_DENSE && c->wfmt != MOE_W_MXFP4) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > 256 || k < 1 || k > 8 || k > E) return MOE_ERR_INVALID_ARG;
+  if (D <= 0 || F <= 0 || D > (1 << 20) || F > (1 << 20)) return MOE_ERR_INVALID_ARG;
+  const int mult = c->wfmt == MOE_W_MXFP4 ? 32 : 16;
+  if (D % mult != 0 || F % mult != 0) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(c->swiglu_limit) || !(c->swiglu_limit > 0.0f) || !std::isfinite(c->swiglu_alpha))
+    return MOE_ERR_INVALID_ARG;
+  if (c->wfmt == MOE_W_MXFP4 && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+bool check_T(int64_t T, int k) { return T >= 0 && T * k < (int64_t(1) << 31); }
+
+size_t elem_size(const moe_config_t* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
+
+size_t ffn_ws_bytes(const moe_config_t* c, int64_t T) {
+  if (c->wfmt != MOE_W_MXFP4 || T == 0) return 0;
+  // dequantised gate and up weights (the down weights reuse the same space)
+  return 2 * align256(size_t(c->num_local_experts) * c->intermediate_size * c->hidden_size * 2);
+}
+
+struct Layout {
+  size_t ids, w, off, ros, sor, pscr, xperm, h, ys, ffn, total;
+};
+
+Layout layout(const moe_config_t* c, int64_t T) {
+  const size_t R = size_t(T) * c->num_experts_per_tok, es = elem_size(c);
+  Layout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.ids = take(R * 4);
+  L.w = take(R * 4);
+  L.off = take(size_t(c->num_local_experts + 1) * 4);
+  L.ros = take(R * 4);
+  L.sor = take(R * 4);
+  L.pscr = take(moe::permute_scratch_words(T, c->num_local_experts) * 4);
+  // x_perm is dead once gate/up has run: the weighted fp32 expert outputs reuse its region
+  L.xperm = take(R * c->hidden_size * (es > 4 ? es : 4));
+  L.ys = L.xperm;
+  L.h = take(R * c->intermediate_size * es);
+  L.ffn = take(ffn_ws_bytes(c, T));
+  L.total = o;
+  return L;
+}
+
+bool get_launch(void* stream, Launch* L) {
+  static std::mutex mu;
+  static int sms[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  int n = 0;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 64 && sms[dev] > 0) {
+      n = sms[dev];
+    } else {
+      if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+      if (dev < 64) sms[dev] = n;
+    }
+  }
+  L->stream = static_cast<cudaStream_t>(stream);
+  L->num_sms = n;
+  L->wait_limit_ns = g_wait_limit_ns.load();
+  return true;
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+bool weights_ok(const moe_config_t* c, const moe_expert_weights_t* w) {
+  if (w == nullptr) return false;
+  if (!ptr_ok(w->w_gate) || !ptr_ok(w->w_up) || !ptr_ok(w->w_down)) return false;
+  if (!ptr_ok(w->b_gate) || !ptr_ok(w->b_up) || !ptr_ok(w->b_down)) return false;
+  if (c->wfmt == MOE_W_MXFP4 && (!ptr_ok(w->s_gate) || !ptr_ok(w->s_up) || !ptr_ok(w->s_down))) return false;
+  return true;
+}
+
+moe::ExpertWeights to_internal(const moe_expert_weights_t* w) {
+  moe::ExpertWeights x;
+  x.w_gate = w->w_gate;
+  x.w_up = w->w_up;
+  x.w_down = w->w_down;
+  x.s_gate = w->s_gate;
+  x.s_up = w->s_up;
+  x.s_down = w->s_down;
+  x.b_gate = w->b_gate;
+  x.b_up = w->b_up;
+  x.b_down = w->b_down;
+  return x;
+}
+
+// gate/up then down (into y_perm, or weighted into slot order when slot_of_row != null)
+moe_status_t run_experts(const moe_config_t* c, const Launch& L, int64_t T, const void* x_perm,
+                         const int32_t* eoff, const moe_expert_weights_t* wts, void* h, void* out,
+                         const int32_t* slot_of_row, const float* topk_w, void* ffn_ws) {
+  const bool bf16 = c->dtype == MOE_BF16;
+  const int D = c->hidden_size, F = c->intermediate_size, E = c->num_local_experts;
+  const int64_t R = T * c->num_experts_per_tok;
+  moe::ExpertWeights w = to_internal(wts);
+  stage_mark(ST_GATEUP, true, L.stream);
+  if (c->wfmt == MOE_W_MXFP4) {
+    uint8_t* buf = static_cast<uint8_t*>(ffn_ws);
+    void* wg = buf;
+    void* wu = buf + align256(size_t(E) * F * D * 2);
+    if (moe::mxfp4_dequant(L, int64_t(E) * F, D, static_cast<const uint8_t*>(wts->w_gate), wts->s_gate, wg) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (moe::mxfp4_dequant(L, int64_t(E) * F, D, static_cast<const uint8_t*>(wts->w_up), wts->s_up, wu) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    w.w_gate = wg;
+    w.w_up = wu;
+    if (moe::expert_gateup(L, true, R, D, F, E, x_perm, eoff, w, c->swiglu_limit, c->swiglu_alpha, h) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    stage_mark(ST_GATEUP, false, L.stream);
+    stage_mark(ST_DOWN, true, L.stream);
+    void* wd = buf;   // gate/up weights are dead once the gate/up kernel (stream-ordered) is done
+    if (moe::mxfp4_dequant(L, int64_t(E) * D, F, static_cast<const uint8_t*>(wts->w_down), wts->s_down, wd) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    w.w_down = wd;
+    const moe_status_t st = cuda_status(moe::expert_down(L, true, R, D, F, E, h, eoff, w, slot_of_row, topk_w, out));
+    stage_mark(ST_DOWN, false, L.stream);
+    return st;
+  }
+  if (moe::expert_gateup(L, bf16, R, D, F, E, x_perm, eoff, w, c->swiglu_limit, c->swiglu_alpha, h) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  stage_mark(ST_GATEUP, false, L.stream);
+  stage_mark(ST_DOWN, true, L.stream);
+  const moe_status_t st = cuda_status(moe::expert_down(L, bf16, R, D, F, E, h, eoff, w, slot_of_row, topk_w, out));
+  stage_mark(ST_DOWN, false, L.stream);
+  return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA call or launch failed";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device wait gave up";
+    case MOE_ERR_DEVICE_BOUNDS: return "MOE_ERR_DEVICE_BOUNDS: out-of-range index read on the device";
+  }
+  return "unknown moe_status_t";
+}
+
+moe_status_t moe_config_check(const moe_config_t* cfg) { return check_cfg(cfg); }
+
+size_t moe_permute_workspace_size(const moe_config_t* cfg, int64_t T) {
+  if (check_cfg(cfg) != MOE_OK || !check_T(T, cfg->num_experts_per_tok)) return size_t(-1);
+  return moe::permute_scratch_words(T, cfg->num_local_experts) * 4;
+}
+
+size_t moe_expert_ffn_workspace_size(const moe_config_t* cfg, int64_t T) {
+  if (check_cfg(cfg) != MOE_OK || !check_T(T, cfg->num_experts_per_tok)) return size_t(-1);
+  return ffn_ws_bytes(cfg, T);
+}
+
+size_t moe_workspace_size(const moe_config_t* cfg, int64_t T) {
+  if (check_cfg(cfg) != MOE_OK || !check_T(T, cfg->num_experts_per_tok)) return size_t(-1);
+  return layout(cfg, T).total;
+}
+
+moe_status_t moe_router_topk(const moe_config_t* cfg, int64_t T, const void* x, const void* w_router,
+                             const void* b_router, int32_t* topk_ids, float* topk_w, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (!check_T(T, cfg->num_experts_per_tok)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!ptr_ok(x) || !ptr_ok(w_router) || !ptr_ok(b_router) || !ptr_ok(topk_ids) || !ptr_ok(topk_w))
+    return MOE_ERR_INVALID_ARG;
+  Launch L;
+  if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
+  return cuda_status(moe::router_topk(L, cfg->dtype == MOE_BF16, T, cfg->hidden_size, cfg->num_local_experts,
+                                      cfg->num_experts_per_tok, x, w_router, b_router, topk_ids, topk_w));
+}
+
+moe_status_t moe_permute(const moe_config_t* cfg, int64_t T, const int32_t* topk_ids, const void* x,
+                         int32_t* expert_off, int32_t* row_of_slot, int32_t* slot_of_row, void* x_perm, void* ws,
+                         size_t ws_bytes, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (!check_T(T, cfg->num_experts_per_tok)) return MOE_ERR_INVALID_ARG;
+  if (!ptr_ok(expert_off)) return MOE_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (!ptr_ok(topk_ids) || !ptr_ok(row_of_slot) || !ptr_ok(slot_of_row)) return MOE_ERR_INVALID_ARG;
+    if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+    if (x != nullptr && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+    const size_t need = moe::permute_scratch_words(T, cfg->num_local_experts) * 4;
+    if (ws == nullptr || !aligned16(ws) || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  }
+  Launch L;
+  if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
+  return cuda_status(moe::permute(L, cfg->dtype == MOE_BF16, T, cfg->hidden_size, cfg->num_local_experts,
+                                  cfg->num_experts_per_tok, topk_ids, x, expert_off, row_of_slot, slot_of_row,
+                                  x_perm, static_cast<int32_t*>(ws)));
+}
+
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, int64_t T, const void* x_perm, const int32_t* expert_off,
+                            const moe_expert_weights_t* weights, void* h, void* y_perm, void* ws, size_t ws_bytes,
+                            void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (!check_T(T, cfg->num_experts_per_tok)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!ptr_ok(x_perm) || !ptr_ok(expert_off) || !ptr_ok(h) || !ptr_ok(y_perm) || !weights_ok(cfg, weights))
+    return MOE_ERR_INVALID_ARG;
+  const size_t need = ffn_ws_bytes(cfg, T);
+  if (need > 0 && (ws == nullptr || !aligned16(ws) || ws_bytes < need)) return MOE_ERR_WORKSPACE;
+  Launch L;
+  if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
+  return run_experts(cfg, L, T, x_perm, expert_off, weights, h, y_perm, nullptr, nullptr, ws);
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, int64_t T, const void* y_perm, const int32_t* row_of_slot,
+                         const float* topk_w, void* y, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (!check_T(T, cfg->num_experts_per_tok)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!ptr_ok(y_perm) || !ptr_ok(row_of_slot) || !ptr_ok(topk_w) || !ptr_ok(y)) return MOE_ERR_INVALID_ARG;
+  Launch L;
+  if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
+  return cuda_status(moe::combine_gather(L, cfg->dtype == MOE_BF16, T, cfg->hidden_size, cfg->num_experts_per_tok,
+                                         y_perm, row_of_slot, topk_w, y));
+}
+
+moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x, const void* w_router,
+                               const void* b_router, const moe_expert_weights_t* weights, void* y,
+                               int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (!check_T(T, cfg->num_experts_per_tok)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!ptr_ok(x) || !ptr_ok(w_router) || !ptr_ok(b_router) || !ptr_ok(y) || !weights_ok(cfg, weights))
+    return MOE_ERR_INVALID_ARG;
+  if ((topk_ids_out != nullptr && !aligned16(topk_ids_out)) || (topk_w_out != nullptr && !aligned16(topk_w_out)))
+    return MOE_ERR_INVALID_ARG;
+  const Layout LY = layout(cfg, T);
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < LY.total) return MOE_ERR_WORKSPACE;
+  Launch L;
+  if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
+
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t*>(base + LY.ids);
+  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(base + LY.w);
+  int32_t* eoff = reinterpret_cast<int32_t*>(base + LY.off);
+  int32_t* ros = reinterpret_cast<int32_t*>(base + LY.ros);
+  int32_t* sor = reinterpret_cast<int32_t*>(base + LY.sor);
+  int32_t* pscr = reinterpret_cast<int32_t*>(base + LY.pscr);
+  void* xperm = base + LY.xperm;
+  void* h = base + LY.h;
+  void* ys = base + LY.ys;
+  void* ffn = base + LY.ffn;
+  const bool bf16 = cfg->dtype == MOE_BF16;
+  const int D = cfg->hidden_size, E = cfg->num_local_experts, k = cfg->num_experts_per_tok;
+
+  stage_mark(ST_ROUTER, true, L.stream);
+  if (moe::router_topk(L, bf16, T, D, E, k, x, w_router, b_router, ids, w) != cudaSuccess) return MOE_ERR_CUDA;
+  stage_mark(ST_ROUTER, false, L.stream);
+  stage_mark(ST_DISPATCH, true, L.stream);
+  if (moe::permute(L, bf16, T, D, E, k, ids, x, eoff, ros, sor, xperm, pscr) != cudaSuccess) return MOE_ERR_CUDA;
+  stage_mark(ST_DISPATCH, false, L.stream);
+  s = run_experts(cfg, L, T, xperm, eoff, weights, h, ys, sor, w, ffn);
+  if (s != MOE_OK) return s;
+  stage_mark(ST_COMBINE, true, L.stream);
+  s = cuda_status(moe::combine_slots(L, bf16, T, D, k, ys, y));
+  stage_mark(ST_COMBINE, false, L.stream);
+  return s;
+}
+
+moe_status_t moe_last_device_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  int bits = 0;
+  if (moe::read_and_clear_device_error(&bits) != cudaSuccess) return MOE_ERR_CUDA;
+  if (bits & moe::DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+  if (bits & moe::DEVERR_BOUNDS) return MOE_ERR_DEVICE_BOUNDS;
+  return MOE_OK;
+}
+
+void moe_set_stage_events(void* const* starts, void* const* stops, int32_t n) {
+  std::lock_guard<std::mutex> g(g_ev_mu);
+  for (int i = 0; i < kStages; ++i) {
+    g_ev_start[i] = (starts != nullptr && i < n) ? static_cast<cudaEvent_t>(starts[i]) : nullptr;
+    g_ev_stop[i] = (stops != nullptr && i < n) ? static_cast<cudaEvent_t>(stops[i]) : nullptr;
+  }
+}
+
+uint64_t moe_launch_count(void) { return moe::g_launches.load(); }
+
+void moe_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns == 0 ? 1000000000ull : ns); }
+
+}  // extern "C"

@@ -1,0 +1,428 @@
+#pragma once
+// Router (SIMT path), dispatch (histogram -> scan -> stable scatter -> row gather),
+// and combine kernels of the GPT-OSS MoE layer.
+//
+// Router: l[t,e] = x[t] . Wr[e] + br[e] (MaxText GPT-OSS weight map, "MoE Router":
+// router kernel + router bias); the k largest logits per token, ties to the lower
+// expert index, and the softmax over the selected k.  This SIMT kernel computes
+// in exact fp32 FMA (no TF32), so fp32 layers route exactly as their definition;
+// bf16 layers with many tokens use the tensor-core router instead.
+//
+// Dispatch: the permutation is the stable sort of the (token, slot) pairs by
+// expert id ("Ollama glm4_moe_lite.go", SwitchMLP.Forward: argsort of the
+// flattened ids, rows gathered from order / k).  It is built without a sort and
+// without order-dependent atomics: per 256-token chunk, every warp builds one
+// 32-bit lane mask per expert (atomicOr is commutative, so the result is
+// deterministic); popcounts give the per-chunk histogram; one scan over
+// (expert, chunk) gives every chunk's base row; a token's row is its base plus the
+// popcount of the lanes before it in its warp and of the warps before it.
+//
+// Combine: y[t] = sum_j w[t,j] * Y[row(t,j)] in fixed j order
+// ("Ollama glm4_moe_lite.go", MoE.Forward: score-weighted sum over the k experts).
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+
+// ---------------------------------------------------------------------------
+// router, SIMT: one block (16 warps) per token
+// ---------------------------------------------------------------------------
+constexpr int kRouterWarps = 16;
+
+template <typename T>
+__device__ __forceinline__ float dot_row16(const T* a, const T* b, int D, int lane) {
+  // 16-byte chunks of both rows, lanes strided over the chunks
+  constexpr int EPC = 16 / sizeof(T);
+  const int nchunk = D / EPC;
+  const uint4* pa = reinterpret_cast<const uint4*>(a);
+  const uint4* pb = reinterpret_cast<const uint4*>(b);
+  float acc = 0.0f;
+  for (int c = lane; c < nchunk; c += 32) {
+    const uint4 ua = pa[c], ub = pb[c];
+    if constexpr (sizeof(T) == 4) {
+      const float* fa = reinterpret_cast<const float*>(&ua);
+      const float* fb = reinterpret_cast<const float*>(&ub);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc = fmaf(fa[i], fb[i], acc);
+    } else {
+      const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&ua);
+      const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&ub);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 fa = __bfloat1622float2(ha[i]);
+        const float2 fb = __bfloat1622float2(hb[i]);
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRouterWarps * 32)
+    router_simt_kernel(const T* __restrict__ x, const T* __restrict__ wr, const T* __restrict__ br, int D, int E,
+                       int k, int32_t* __restrict__ ids, float* __restrict__ wout) {
+  __shared__ float logits[256];
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const T* xr = x + static_cast<size_t>(t) * D;
+  for (int e = warp; e < E; e += kRouterWarps) {
+    const float l = dot_row16<T>(xr, wr + static_cast<size_t>(e) * D, D, lane);
+    if (lane == 0) logits[e] = l + to_f32<T>(br[e]);
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  // each lane holds experts lane, lane+32, ... (E <= 256 -> 8 values)
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? logits[e] : -INFINITY;
+  }
+  float sel_v[8];
+  int sel_e[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    sel_v[j] = -INFINITY;
+    sel_e[j] = -1;
+    if (j < k) {
+      // lane-local best: larger value, then lower expert index
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && (v[i] > bv || (v[i] == bv && e < be))) { bv = v[i]; be = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+      }
+      sel_v[j] = bv;
+      sel_e[j] = be;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i == be) v[i] = -INFINITY;
+    }
+  }
+  if (lane == 0) {
+    float z = 0.0f, ex[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      ex[j] = j < k ? expf(sel_v[j] - sel_v[0]) : 0.0f;
+      z += ex[j];
+    }
+    const float inv = 1.0f / z;
+    for (int j = 0; j < k; ++j) {
+      ids[static_cast<size_t>(t) * k + j] = sel_e[j];
+      wout[static_cast<size_t>(t) * k + j] = ex[j] * inv;
+    }
+  }
+}
+
+cudaError_t router_tc(const Launch& L, int64_t T, int D, int E, int k, const void* x, const void* w_router,
+                      const void* b_router, int32_t* ids, float* w);   // gemm_launch.cu
+
+cudaError_t router_topk(const Launch& L, bool bf16, int64_t T, int D, int E, int k, const void* x,
+                        const void* w_router, const void* b_router, int32_t* ids, float* w) {
+  if (T == 0) return cudaSuccess;
+  if (bf16 && T >= 256) return router_tc(L, T, D, E, k, x, w_router, b_router, ids, w);
+  const dim3 grid(static_cast<unsigned>(T));
+  if (bf16)
+    router_simt_kernel<__nv_bfloat16><<<grid, kRouterWarps * 32, 0, L.stream>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
+        static_cast<const __nv_bfloat16*>(b_router), D, E, k, ids, w);
+  else
+    router_simt_kernel<float><<<grid, kRouterWarps * 32, 0, L.stream>>>(
+        static_cast<const float*>(x), static_cast<const float*>(w_router), static_cast<const float*>(b_router), D,
+        E, k, ids, w);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// dispatch
+// ---------------------------------------------------------------------------
+constexpr int kChunk = 256;   // tokens per chunk = 8 warps x 32 lanes
+constexpr int kChunkWarps = kChunk / 32;
+
+size_t permute_scratch_words(int64_t T, int E) {
+  const int64_t nchunks = (T + kChunk - 1) / kChunk;
+  return static_cast<size_t>(2 * nchunks * E);
+}
+
+// Build the per-warp expert lane masks of one chunk.  Returns false (and flags the
+// device error word) if an id is out of range or repeated within a token.
+__device__ __forceinline__ void build_masks(uint32_t (*mask)[256], const int32_t* __restrict__ ids, int T, int k,
+                                            int E) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kChunkWarps * 256; i += blockDim.x) (&mask[0][0])[i] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kChunk + threadIdx.x;
+  if (t < T) {
+    int prev[8];
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[static_cast<size_t>(t) * k + j];
+      bool bad = e < 0 || e >= E;
+      for (int q = 0; q < j && q < 8; ++q) bad |= (prev[q] == e);
+      if (j < 8) prev[j] = e;
+      if (bad) {
+        flag_error(DEVERR_BOUNDS);
+        continue;
+      }
+      atomicOr(&mask[warp][e], 1u << lane);
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kChunk) permute_count_kernel(const int32_t* __restrict__ ids, int T, int k, int E,
+                                                               int nchunks, int32_t* __restrict__ chunk_cnt) {
+  __shared__ uint32_t mask[kChunkWarps][256];
+  build_masks(mask, ids, T, k, E);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kChunkWarps; ++w) c += __popc(mask[w][e]);
+    chunk_cnt[static_cast<size_t>(e) * nchunks + blockIdx.x] = c;
+  }
+}
+
+// Exclusive scan over the expert-major (expert, chunk) counts; one block.
+__global__ void __launch_bounds__(1024) permute_scan_kernel(const int32_t* __restrict__ cnt, int n, int E, int nchunks,
+                                                            int32_t* __restrict__ base, int32_t* __restrict__ expert_off) {
+  __shared__ int warp_tot[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int b = min(n, tid * per), e = min(n, b + per);
+  int local = 0;
+  for (int i = b; i < e; ++i) local += cnt[i];
+  int incl = local;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int v = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, v, d);
+      if (lane >= d) v += o;
+    }
+    if (lane < nw) warp_tot[lane] = v;   // inclusive
+  }
+  __syncthreads();
+  int run = incl - local + (warp > 0 ? warp_tot[warp - 1] : 0);
+  for (int i = b; i < e; ++i) {
+    base[i] = run;
+    run += cnt[i];
+  }
+  __syncthreads();
+  for (int q = tid; q < E; q += blockDim.x) expert_off[q] = base[static_cast<size_t>(q) * nchunks];
+  if (tid == blockDim.x - 1) expert_off[E] = warp_tot[(blockDim.x >> 5) - 1];
+}
+
+__global__ void __launch_bounds__(kChunk) permute_scatter_kernel(const int32_t* __restrict__ ids, int T, int k, int E,
+                                                                 int nchunks, const int32_t* __restrict__ base,
+                                                                 int32_t* __restrict__ row_of_slot,
+                                                                 int32_t* __restrict__ slot_of_row) {
+  __shared__ uint32_t mask[kChunkWarps][256];
+  build_masks(mask, ids, T, k, E);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kChunk + threadIdx.x;
+  if (t >= T) return;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int R = T * k;
+  for (int j = 0; j < k; ++j) {
+    const int e = ids[static_cast<size_t>(t) * k + j];
+    if (e < 0 || e >= E) continue;
+    int r = base[static_cast<size_t>(e) * nchunks + blockIdx.x] + __popc(mask[warp][e] & lt);
+    for (int w = 0; w < warp; ++w) r += __popc(mask[w][e]);
+    if (r < 0 || r >= R) {
+      flag_error(DEVERR_BOUNDS);
+      continue;
+    }
+    row_of_slot[static_cast<size_t>(t) * k + j] = r;
+    slot_of_row[r] = t * k + j;
+  }
+}
+
+// x_perm[r] = x[slot_of_row[r] / k], one warp per row, 16-byte vectors.
+__global__ void permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ slot_of_row, int R,
+                                      int k, int T, int vec_per_row, uint4* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int r = gw; r < R; r += nw) {
+    const int s = slot_of_row[r];
+    const int t = s / k;
+    if (s < 0 || t >= T) {
+      if (lane == 0) flag_error(DEVERR_BOUNDS);
+      continue;
+    }
+    const uint4* src = x + static_cast<size_t>(t) * vec_per_row;
+    uint4* dst = x_perm + static_cast<size_t>(r) * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+  }
+}
+
+cudaError_t permute(const Launch& L, bool bf16, int64_t T, int D, int E, int k, const int32_t* ids, const void* x,
+                    int32_t* expert_off, int32_t* row_of_slot, int32_t* slot_of_row, void* x_perm,
+                    int32_t* scratch) {
+  if (T == 0) {
+    return cudaMemsetAsync(expert_off, 0, sizeof(int32_t) * (E + 1), L.stream);
+  }
+  const int nchunks = static_cast<int>((T + kChunk - 1) / kChunk);
+  int32_t* cnt = scratch;
+  int32_t* base = scratch + static_cast<size_t>(nchunks) * E;
+  permute_count_kernel<<<nchunks, kChunk, 0, L.stream>>>(ids, static_cast<int>(T), k, E, nchunks, cnt);
+  permute_scan_kernel<<<1, 1024, 0, L.stream>>>(cnt, nchunks * E, E, nchunks, base, expert_off);
+  permute_scatter_kernel<<<nchunks, kChunk, 0, L.stream>>>(ids, static_cast<int>(T), k, E, nchunks, base,
+                                                           row_of_slot, slot_of_row);
+  count_launch(3);
+  if (x != nullptr && x_perm != nullptr) {
+    const int R = static_cast<int>(T * k);
+    const int vpr = D * (bf16 ? 2 : 4) / 16;
+    const int warps_needed = R;
+    const int blocks = static_cast<int>(std::min<int64_t>((warps_needed + 7) / 8, int64_t(L.num_sms) * 8));
+    permute_gather_kernel<<<blocks, 256, 0, L.stream>>>(static_cast<const uint4*>(x), slot_of_row, R, k,
+                                                       static_cast<int>(T), vpr, static_cast<uint4*>(x_perm));
+    count_launch();
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// combine
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void combine_gather_kernel(const T* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
+                                      const float* __restrict__ w, int Tn, int k, int D, T* __restrict__ y) {
+  const int nv = D / 8;
+  const int64_t total = static_cast<int64_t>(Tn) * nv;
+  const int R = Tn * k;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(i / nv);
+    const int c = static_cast<int>(i - static_cast<int64_t>(t) * nv) * 8;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < k; ++j) {
+      const int r = row_of_slot[static_cast<size_t>(t) * k + j];
+      if (r < 0 || r >= R) {
+        flag_error(DEVERR_BOUNDS);
+        continue;
+      }
+      const float wt = w[static_cast<size_t>(t) * k + j];
+      float v[8];
+      load8<T>(y_perm + static_cast<size_t>(r) * D + c, v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = fmaf(wt, v[q], acc[q]);
+    }
+    store8<T>(y + static_cast<size_t>(t) * D + c, acc);
+  }
+}
+
+template <typename T>
+__global__ void combine_slots_kernel(const float* __restrict__ ys, int Tn, int k, int D, T* __restrict__ y) {
+  const int nv = D / 8;
+  const int64_t total = static_cast<int64_t>(Tn) * nv;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(i / nv);
+    const int c = static_cast<int>(i - static_cast<int64_t>(t) * nv) * 8;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < k; ++j) {
+      float v[8];
+      load8<float>(ys + (static_cast<size_t>(t) * k + j) * D + c, v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] += v[q];
+    }
+    store8<T>(y + static_cast<size_t>(t) * D + c, acc);
+  }
+}
+
+static int elementwise_blocks(const Launch& L, int64_t items) {
+  const int64_t want = (items + 255) / 256;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(L.num_sms) * 16)));
+}
+
+cudaError_t combine_gather(const Launch& L, bool bf16, int64_t T, int D, int k, const void* y_perm,
+                           const int32_t* row_of_slot, const float* w, void* y) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = elementwise_blocks(L, T * (D / 8));
+  if (bf16)
+    combine_gather_kernel<__nv_bfloat16><<<blocks, 256, 0, L.stream>>>(
+        static_cast<const __nv_bfloat16*>(y_perm), row_of_slot, w, static_cast<int>(T), k, D,
+        static_cast<__nv_bfloat16*>(y));
+  else
+    combine_gather_kernel<float><<<blocks, 256, 0, L.stream>>>(static_cast<const float*>(y_perm), row_of_slot, w,
+                                                              static_cast<int>(T), k, D, static_cast<float*>(y));
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t combine_slots(const Launch& L, bool bf16, int64_t T, int D, int k, const void* ys, void* y) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = elementwise_blocks(L, T * (D / 8));
+  if (bf16)
+    combine_slots_kernel<__nv_bfloat16><<<blocks, 256, 0, L.stream>>>(
+        static_cast<const float*>(ys), static_cast<int>(T), k, D, static_cast<__nv_bfloat16*>(y));
+  else
+    combine_slots_kernel<float><<<blocks, 256, 0, L.stream>>>(static_cast<const float*>(ys), static_cast<int>(T),
+                                                             k, D, static_cast<float*>(y));
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// MXFP4 -> bf16 (E2M1 code: sign bit 3, exponent bits 2..1 with bias 1, mantissa bit 0;
+// E8M0 scale 2^(s-127) per 32 elements; element 2i = low nibble of byte i)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float e2m1_to_float(uint32_t c) {
+  const uint32_t ex = (c >> 1) & 3u, man = c & 1u;
+  const float mag = ex == 0 ? 0.5f * static_cast<float>(man) : ldexpf(1.0f + 0.5f * static_cast<float>(man), ex - 1);
+  return (c & 8u) ? -mag : mag;
+}
+
+__global__ void mxfp4_dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ s, int64_t rows, int K,
+                                     __nv_bfloat16* __restrict__ out) {
+  const int64_t total = rows * (K / 2);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / (K / 2);
+    const int b = static_cast<int>(i - r * (K / 2));
+    const uint32_t byte = q[i];
+    const float sc = ldexpf(1.0f, static_cast<int>(s[r * (K / 32) + (2 * b) / 32]) - 127);
+    out[r * K + 2 * b] = __float2bfloat16_rn(e2m1_to_float(byte & 0xFu) * sc);
+    out[r * K + 2 * b + 1] = __float2bfloat16_rn(e2m1_to_float(byte >> 4) * sc);
+  }
+}
+
+cudaError_t mxfp4_dequant(const Launch& L, int64_t rows, int K, const uint8_t* q, const uint8_t* s, void* out) {
+  if (rows == 0) return cudaSuccess;
+  const int blocks = elementwise_blocks(L, rows * (K / 2));
+  mxfp4_dequant_kernel<<<blocks, 256, 0, L.stream>>>(q, s, rows, K, static_cast<__nv_bfloat16*>(out));
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error(int* bits) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  *bits = v;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+}
+
+}  // namespace moe

@@ -214,21 +214,19 @@ def layer_tokens(layer: Dict[str, np.ndarray], tokens: np.ndarray, k: int, limit
     ids, w = topk_softmax(logits, k)
     D = layer["b_down"].shape[1]
     F = layer["b_gate"].shape[1]
-    y = np.zeros((tokens.size, D))
     h = np.zeros((tokens.size, k, F))
-    cache: Dict[int, Tuple[np.ndarray, np.ndarray, np.ndarray]] = {}
-    for i in range(tokens.size):
-        for j in range(k):
-            e = int(ids[i, j])
-            if e not in cache:
-                cache[e] = (expert_weights(layer, "gate", e), expert_weights(layer, "up", e),
-                            expert_weights(layer, "down", e))
-                if len(cache) > 8:
-                    cache.pop(next(iter(cache)))
-            wg, wu, wd = cache[e]
-            g = wg @ x[i] + decode(layer["b_gate"][e])
-            u = wu @ x[i] + decode(layer["b_up"][e])
-            hh = clipped_swiglu(g, u, limit, alpha)
-            h[i, j] = hh
-            y[i] += w[i, j] * (wd @ hh + decode(layer["b_down"][e]))
+    o = np.zeros((tokens.size, k, D))
+    # each selected expert's weights are decoded once, for all the tokens that chose it
+    for e in np.unique(ids):
+        e = int(e)
+        ii, jj = np.nonzero(ids == e)
+        xs = x[ii]
+        g = xs @ expert_weights(layer, "gate", e).T + decode(layer["b_gate"][e])
+        u = xs @ expert_weights(layer, "up", e).T + decode(layer["b_up"][e])
+        hh = clipped_swiglu(g, u, limit, alpha)
+        h[ii, jj] = hh
+        o[ii, jj] = hh @ expert_weights(layer, "down", e).T + decode(layer["b_down"][e])
+    y = np.zeros((tokens.size, D))
+    for j in range(k):
+        y += w[:, j:j + 1] * o[:, j]
     return dict(logits=logits, ids=ids, w=w, h=h, y=y)

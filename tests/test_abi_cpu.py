@@ -1,0 +1,126 @@
+"""The C-ABI library loads and exports every symbol include/moe.h declares, and
+its host-side validation rejects bad arguments before touching the GPU.
+No compute call is made here (these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+from mixture_experts_ffn_12_b200 import _lib, build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src, flags=re.M)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_lib.SIGNATURES), "binding signatures must cover exactly the header"
+
+
+def test_struct_layout_matches_header():
+    assert ctypes.sizeof(_lib.MoeConfig) == 32
+    assert ctypes.sizeof(_lib.MoeExpertWeights) == 9 * ctypes.sizeof(ctypes.c_void_p)
+
+
+def cfg(**kw):
+    base = dict(hidden_size=2880, intermediate_size=2880, num_local_experts=32, num_experts_per_tok=4,
+                swiglu_limit=7.0, swiglu_alpha=1.702, dtype=_lib.MOE_BF16, wfmt=_lib.MOE_W_DENSE)
+    base.update(kw)
+    return _lib.MoeConfig(**base)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.moe_abi_version() == 1
+    for code in range(7):
+        assert lib.moe_status_string(code).startswith(b"MOE_")
+    assert b"unknown" in lib.moe_status_string(99)
+
+
+@pytest.mark.parametrize("kw,want", [
+    ({}, _lib.MOE_OK),
+    (dict(dtype=_lib.MOE_F32, hidden_size=256, intermediate_size=512, num_local_experts=8, num_experts_per_tok=2),
+     _lib.MOE_OK),
+    (dict(wfmt=_lib.MOE_W_MXFP4), _lib.MOE_OK),
+    (dict(wfmt=_lib.MOE_W_MXFP4, dtype=_lib.MOE_F32), _lib.MOE_ERR_UNSUPPORTED),
+    (dict(num_experts_per_tok=0), _lib.MOE_ERR_INVALID_ARG),
+    (dict(num_experts_per_tok=9, num_local_experts=16), _lib.MOE_ERR_INVALID_ARG),
+    (dict(num_experts_per_tok=5, num_local_experts=4), _lib.MOE_ERR_INVALID_ARG),
+    (dict(num_local_experts=257), _lib.MOE_ERR_INVALID_ARG),
+    (dict(hidden_size=2888), _lib.MOE_ERR_INVALID_ARG),                 # not a multiple of 16
+    (dict(wfmt=_lib.MOE_W_MXFP4, intermediate_size=2896), _lib.MOE_ERR_INVALID_ARG),  # not a multiple of 32
+    (dict(hidden_size=0), _lib.MOE_ERR_INVALID_ARG),
+    (dict(swiglu_limit=0.0), _lib.MOE_ERR_INVALID_ARG),
+    (dict(swiglu_limit=float("inf")), _lib.MOE_ERR_INVALID_ARG),
+    (dict(swiglu_limit=float("nan")), _lib.MOE_ERR_INVALID_ARG),
+    (dict(dtype=7), _lib.MOE_ERR_INVALID_ARG),
+    (dict(wfmt=3), _lib.MOE_ERR_INVALID_ARG),
+])
+def test_config_check(lib, kw, want):
+    assert lib.moe_config_check(ctypes.byref(cfg(**kw))) == want
+
+
+def test_null_config(lib):
+    assert lib.moe_config_check(None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_workspace_size(None, 4) == _lib.SIZE_INVALID
+
+
+def test_workspace_sizes(lib):
+    c = cfg()
+    assert lib.moe_permute_workspace_size(ctypes.byref(c), 0) == 0
+    assert lib.moe_expert_ffn_workspace_size(ctypes.byref(c), 4096) == 0
+    T, k, D, F = 4096, 4, 2880, 2880
+    ws = lib.moe_workspace_size(ctypes.byref(c), T)
+    R = T * k
+    # x_perm's region holds the fp32 weighted outputs later (R*D*4), then h, plus maps
+    assert ws >= R * D * 4 + R * F * 2 + 4 * R * 4
+    assert ws < R * D * 4 + R * F * 2 + 4 * R * 4 + 64 * 1024 * 1024
+    assert lib.moe_workspace_size(ctypes.byref(c), -1) == _lib.SIZE_INVALID
+    assert lib.moe_workspace_size(ctypes.byref(c), 1 << 30) == _lib.SIZE_INVALID   # T*k >= 2^31
+    mx = cfg(wfmt=_lib.MOE_W_MXFP4)
+    assert lib.moe_expert_ffn_workspace_size(ctypes.byref(mx), 8) >= 2 * 32 * 2880 * 2880 * 2
+
+
+def test_rejections_launch_nothing(lib):
+    """Every one of these returns before any CUDA call (no GPU here)."""
+    c = cfg()
+    p = ctypes.c_void_p(0x10000)        # aligned, never dereferenced
+    bad = ctypes.c_void_p(0x10008)      # misaligned
+    assert lib.moe_router_topk(ctypes.byref(c), 0, None, None, None, None, None, None) == _lib.MOE_OK
+    assert lib.moe_router_topk(ctypes.byref(c), 8, None, p, p, p, p, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_topk(ctypes.byref(c), 8, bad, p, p, p, p, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_topk(ctypes.byref(c), -1, p, p, p, p, p, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_topk(None, 8, p, p, p, p, p, None) == _lib.MOE_ERR_INVALID_ARG
+    # permute: workspace too small, x without x_perm
+    assert lib.moe_permute(ctypes.byref(c), 8, p, p, p, p, p, p, p, 0, None) == _lib.MOE_ERR_WORKSPACE
+    assert lib.moe_permute(ctypes.byref(c), 8, p, p, p, p, p, None, p, 1 << 20, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute(ctypes.byref(c), 8, p, p, None, p, p, p, p, 1 << 20, None) == _lib.MOE_ERR_INVALID_ARG
+    w = _lib.MoeExpertWeights(*([0x10000] * 3 + [None] * 3 + [0x10000] * 3))
+    assert lib.moe_expert_ffn(ctypes.byref(c), 8, p, p, None, p, p, None, 0, None) == _lib.MOE_ERR_INVALID_ARG
+    # MXFP4 needs scales and a workspace
+    mx = cfg(wfmt=_lib.MOE_W_MXFP4)
+    assert lib.moe_expert_ffn(ctypes.byref(mx), 8, p, p, ctypes.byref(w), p, p, None, 0, None) == \
+        _lib.MOE_ERR_INVALID_ARG
+    wmx = _lib.MoeExpertWeights(*([0x10000] * 9))
+    assert lib.moe_expert_ffn(ctypes.byref(mx), 8, p, p, ctypes.byref(wmx), p, p, None, 0, None) == \
+        _lib.MOE_ERR_WORKSPACE
+    assert lib.moe_combine(ctypes.byref(c), 8, p, None, p, p, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_forward(ctypes.byref(c), 8, p, p, p, ctypes.byref(w), p, None, None, p, 10, None) == \
+        _lib.MOE_ERR_WORKSPACE
+    assert lib.moe_layer_forward(ctypes.byref(c), 8, p, p, p, None, p, None, None, p, 1 << 40, None) == \
+        _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_forward(ctypes.byref(c), 0, None, None, None, None, None, None, None, None, 0, None) == \
+        _lib.MOE_OK

@@ -1,0 +1,228 @@
+"""CUDA path vs the CPU oracle, through the C ABI (all marked gpu).
+
+Bit-exact: expert ids (as sets; slot order where the logits are separated),
+the dispatch maps and x_perm.  Floating point: max |got - ref| / RMS(ref) of
+the layer output <= 2e-2 (bf16 and fp32 layers) or 5e-2 (MXFP4), the
+acceptance bounds of the layer; the intermediates h and y_perm, which are
+stored in the activation dtype, get the same bound plus their storage rounding
+(2^-8 |ref| per element for bf16); routing weights within 2e-5.
+Full-size layers are compared on every routing decision and on a sample of
+token outputs that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import moe_oracle as O
+from parity_util import TOL_W, check_ids, check_stored, f64, layer_for, rel_rms, tol_for
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def api(cuda_ok):
+    from mixture_experts_ffn_12_b200 import api as A, build
+    build.build()
+    return A
+
+
+RAGGED_BF16 = W.tiny_spec(T=300, D=128, E=7, k=2, F=272, dtype="bf16", cfg_id=201)
+RAGGED_F32 = W.tiny_spec(T=77, D=96, E=5, k=3, F=144, dtype="f32", cfg_id=202)
+WIDE_K = W.tiny_spec(T=260, D=64, E=16, k=8, F=48, dtype="bf16", cfg_id=203)
+ONE_EXPERT = W.tiny_spec(T=40, D=32, E=1, k=1, F=32, dtype="bf16", cfg_id=204)
+MXFP4_SMALL = W.tiny_spec(T=280, D=128, E=6, k=2, F=160, dtype="bf16", wfmt="mxfp4", cfg_id=205)
+
+SMALL_SPECS = [W.TINY_FP32, RAGGED_BF16, RAGGED_F32, WIDE_K, ONE_EXPERT, MXFP4_SMALL]
+DECODE_SPECS = [W.gptoss20b_decode(t) for t in W.GPTOSS20B_DECODE_T]
+
+
+def dev(layer, api):
+    return api.upload_layer(layer)
+
+
+# --------------------------------------------------------------------------- #
+# router + top-k
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("spec", SMALL_SPECS + [W.GPTOSS20B_PREFILL, W.gptoss20b_decode(8), W.GPTOSS120B_SKEWED],
+                         ids=lambda s: s.name)
+def test_router_topk(api, spec):
+    layer = layer_for(spec, experts=False)
+    d = dev({k: layer[k] for k in ("x", "w_router", "b_router")}, api)
+    cfg = api.config_from_spec(spec)
+    ids, w = api.router_topk(cfg, d["x"], d["w_router"], d["b_router"])
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    lg = O.router_logits(layer["x"], layer["w_router"], layer["b_router"])
+    rid, rw = O.topk_softmax(lg, spec.k)
+    gid = ids.cpu().numpy()
+    check_ids(gid, rid, lg)
+    # weights: compare on the oracle's order (same sets)
+    gw = w.cpu().numpy().astype(np.float64)
+    order_map = np.argsort(gid, axis=1)
+    ref_sorted = np.take_along_axis(rw, np.argsort(rid, axis=1), axis=1)
+    got_sorted = np.take_along_axis(gw, order_map, axis=1)
+    assert np.max(np.abs(got_sorted - ref_sorted)) <= TOL_W
+    np.testing.assert_allclose(gw.sum(axis=1), 1.0, atol=1e-6)
+
+
+# --------------------------------------------------------------------------- #
+# dispatch
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("T,E,k,D", [(1, 1, 1, 16), (5, 4, 2, 32), (257, 256, 8, 16), (1000, 3, 3, 48),
+                                     (4096, 32, 4, 64), (70000, 128, 4, 16)])
+def test_permute_bit_exact(api, T, E, k, D):
+    rng = np.random.default_rng(T + E)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    x = rng.standard_normal((T, D)).astype(np.float32)
+    cfg = api.make_config(D, 32, E, k, dtype="f32")
+    out = api.permute(cfg, torch.from_numpy(ids).cuda(), torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    off, ros, sor = O.dispatch(ids, E)
+    assert np.array_equal(out["expert_off"].cpu().numpy(), off)
+    assert np.array_equal(out["row_of_slot"].cpu().numpy(), ros)
+    assert np.array_equal(out["slot_of_row"].cpu().numpy(), sor)
+    assert np.array_equal(out["x_perm"].cpu().numpy(), O.permute_rows(x, sor, k))
+
+
+def test_permute_empty_and_index_only(api):
+    cfg = api.make_config(32, 32, 4, 2, dtype="bf16")
+    out = api.permute(cfg, torch.zeros((0, 2), dtype=torch.int32, device="cuda"))
+    assert out["expert_off"].cpu().numpy().tolist() == [0] * 5
+    ids = torch.tensor([[1, 0], [1, 3], [3, 2]], dtype=torch.int32, device="cuda")
+    out = api.permute(cfg, ids)
+    torch.cuda.synchronize()
+    assert out["expert_off"].cpu().numpy().tolist() == [0, 1, 3, 4, 6]
+    assert out["slot_of_row"].cpu().numpy().tolist() == [1, 0, 2, 5, 3, 4]
+
+
+def test_permute_bad_ids_flag_device_error(api):
+    from mixture_experts_ffn_12_b200 import _lib
+    cfg = api.make_config(32, 32, 4, 2, dtype="bf16")
+    ids = torch.tensor([[1, 7], [2, 2]], dtype=torch.int32, device="cuda")   # out of range; repeated
+    api.permute(cfg, ids, torch.zeros((2, 32), dtype=torch.bfloat16, device="cuda"))
+    assert api.last_device_error() == _lib.MOE_ERR_DEVICE_BOUNDS
+    assert api.last_device_error() == 0                                        # cleared, context usable
+
+
+# --------------------------------------------------------------------------- #
+# expert FFN (gate/up + SwiGLU, down) and combine, from the oracle's dispatch
+# --------------------------------------------------------------------------- #
+def _expert_inputs(spec, layer, api):
+    lg = O.router_logits(layer["x"], layer["w_router"], layer["b_router"])
+    ids, w = O.topk_softmax(lg, spec.k)
+    off, ros, sor = O.dispatch(ids, spec.E)
+    xp = layer["x"][sor // spec.k]                          # permuted rows, storage format
+    return ids, w, off, ros, sor, xp
+
+
+@pytest.mark.parametrize("spec", SMALL_SPECS, ids=lambda s: s.name)
+def test_expert_ffn(api, spec):
+    layer = layer_for(spec)
+    ids, w, off, ros, sor, xp = _expert_inputs(spec, layer, api)
+    d = dev({k: v for k, v in layer.items() if k not in ("x",)}, api)
+    cfg = api.config_from_spec(spec)
+    h, yp = api.expert_ffn(cfg, api.to_torch(xp).cuda(), torch.from_numpy(off).cuda(), api.expert_weights_from(d))
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    rh, ry = O.expert_ffn(xp, off, layer, spec.limit, spec.alpha)
+    tol = tol_for(spec)
+    check_stored(f64(h), rh, tol, spec.dtype == "bf16")
+    check_stored(f64(yp), ry, tol, spec.dtype == "bf16")
+
+
+@pytest.mark.parametrize("spec", [W.GPTOSS20B_PREFILL], ids=lambda s: s.name)
+def test_expert_ffn_full_size_some_experts(api, spec):
+    """GPT-OSS-20B-shaped gate/up/down on all 16384 routed rows; the oracle checks three whole experts."""
+    layer = layer_for(spec)
+    ids, w, off, ros, sor, xp = _expert_inputs(spec, layer, api)
+    d = dev({k: v for k, v in layer.items() if k not in ("x",)}, api)
+    cfg = api.config_from_spec(spec)
+    h, yp = api.expert_ffn(cfg, api.to_torch(xp).cuda(), torch.from_numpy(off).cuda(), api.expert_weights_from(d))
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    for e in (0, 13, spec.E - 1):
+        a, b = int(off[e]), int(off[e + 1])
+        sub = dict(layer)
+        sub_off = np.zeros(spec.E + 1, np.int32)
+        sub_off[e + 1:] = b - a
+        rh, ry = O.expert_ffn(xp[a:b], sub_off, sub, spec.limit, spec.alpha)
+        check_stored(f64(h[a:b]), rh, 2e-2, True)
+        check_stored(f64(yp[a:b]), ry, 2e-2, True)
+
+
+@pytest.mark.parametrize("spec", [W.TINY_FP32, RAGGED_BF16, WIDE_K], ids=lambda s: s.name)
+def test_combine(api, spec):
+    rng = np.random.default_rng(11)
+    T, k, D = spec.T, spec.k, spec.D
+    ids = np.stack([rng.permutation(spec.E)[:k] for _ in range(T)]).astype(np.int32)
+    _, ros, _ = O.dispatch(ids, spec.E)
+    w = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
+    yp = rng.standard_normal((T * k, D)).astype(np.float32)
+    if spec.dtype == "bf16":
+        yp_store = W.f32_to_bf16_bits(yp)
+    else:
+        yp_store = yp
+    cfg = api.config_from_spec(spec)
+    y = api.combine(cfg, api.to_torch(yp_store).cuda(), torch.from_numpy(ros).cuda(), torch.from_numpy(w).cuda())
+    ref = O.combine(O.decode(yp_store), ros, w.astype(np.float64))
+    assert rel_rms(f64(y), ref) <= (1e-2 if spec.dtype == "bf16" else 1e-6)
+
+
+# --------------------------------------------------------------------------- #
+# whole layer
+# --------------------------------------------------------------------------- #
+def _run_layer(api, spec, layer):
+    d = dev(layer, api)
+    cfg = api.config_from_spec(spec)
+    ids = torch.empty((spec.T, spec.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((spec.T, spec.k), dtype=torch.float32, device="cuda")
+    y = api.layer_forward(cfg, d["x"], d["w_router"], d["b_router"], api.expert_weights_from(d),
+                          topk_ids=ids, topk_w=w)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    return y, ids.cpu().numpy(), w
+
+
+@pytest.mark.parametrize("spec", SMALL_SPECS + DECODE_SPECS, ids=lambda s: s.name)
+def test_layer_forward_all_tokens(api, spec):
+    layer = layer_for(spec)
+    y, gid, _ = _run_layer(api, spec, layer)
+    ref = O.layer_tokens(layer, np.arange(spec.T), spec.k, spec.limit, spec.alpha)
+    check_ids(gid, ref["ids"], ref["logits"])
+    assert rel_rms(f64(y), ref["y"]) <= tol_for(spec)
+
+
+@pytest.mark.parametrize("spec", [W.GPTOSS20B_PREFILL, W.GPTOSS20B_MXFP4, W.GPTOSS120B_SKEWED],
+                         ids=lambda s: s.name)
+def test_layer_forward_full_size_sampled(api, spec):
+    layer = layer_for(spec)
+    y, gid, _ = _run_layer(api, spec, layer)
+    # routing: every token, bit-exact
+    lg = O.router_logits(layer["x"], layer["w_router"], layer["b_router"])
+    rid, _ = O.topk_softmax(lg, spec.k)
+    check_ids(gid, rid, lg)
+    off, _, sor = O.dispatch(rid, spec.E)
+    # outputs: a sample that covers the first and last tokens and the busiest expert
+    rng = np.random.default_rng(5)
+    toks = np.unique(np.concatenate([[0, spec.T - 1], rng.choice(spec.T, 46, replace=False),
+                                     sor[off[0]:off[1]][:16] // spec.k]))
+    ref = O.layer_tokens(layer, toks, spec.k, spec.limit, spec.alpha)
+    got = f64(y[torch.from_numpy(toks).cuda()])
+    # the RMS of the full output, estimated from the sample
+    assert rel_rms(got, ref["y"]) <= tol_for(spec)
+
+
+def test_layer_forward_repeatable(api):
+    """Two calls on the same inputs give bit-identical outputs (no order-dependent atomics)."""
+    spec = RAGGED_BF16
+    layer = layer_for(spec)
+    d = dev(layer, api)
+    cfg = api.config_from_spec(spec)
+    ew = api.expert_weights_from(d)
+    y1 = api.layer_forward(cfg, d["x"], d["w_router"], d["b_router"], ew)
+    y2 = api.layer_forward(cfg, d["x"], d["w_router"], d["b_router"], ew)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
