@@ -48,6 +48,7 @@ def parse_args():
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default="gptoss20b_prefill", choices=sorted(W.SPECS))
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-decode", action="store_true", help="skip the decode-regime sweep")
     return p.parse_args()
 
 
@@ -299,6 +300,8 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1))
 
+    decode = decode_sweep(api, moe, spec, layer, dev, stream, max(20, K // 4)) if not args.no_decode else None
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(spec, layer)
@@ -332,11 +335,46 @@ def run_ours(args, rank, world, local_rank):
             "gpu_launches": int(launches),
             "clocks": sampler.summary(),
         }
+        if decode is not None:
+            line["decode"] = decode
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def decode_sweep(api, moe, spec, layer, dev, stream, steps):
+    """Decode regime of the same layer (T = 1, 8, 32, 64): GB/s of the expert weights the step touches.
+
+    Touched bytes = (experts with at least one routed token) x 3 x D x F x element size, plus the
+    router weights; each step streams them from HBM (T = 1 touches 4 experts = 0.2 GB > L2).
+    """
+    import torch
+    peaks = measured_peaks()
+    out = {}
+    esz = 2 if spec.dtype == "bf16" else 4
+    for T in W.GPTOSS20B_DECODE_T:
+        dspec = W.gptoss20b_decode(T) if spec.name.startswith("gptoss20b") else spec.with_tokens(T)
+        x = api.to_torch(W.make_layer(dspec, seed=0, with_experts=False)["x"]).to(dev)
+        y = torch.empty_like(x)
+        ids = torch.empty((T, spec.k), dtype=torch.int32, device=dev)
+        for _ in range(5):
+            moe(x, y=y, topk_ids=ids)
+        torch.cuda.synchronize()
+        touched = int(torch.unique(ids).numel())
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            moe(x, y=y, topk_ids=ids)
+        b.record(stream)
+        torch.cuda.synchronize()
+        us = 1e3 * a.elapsed_time(b) / steps
+        nbytes = touched * 3 * spec.D * spec.F * esz + spec.E * spec.D * esz
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[f"T{T}"] = {"us_per_step": us, "experts_touched": touched, "weight_bytes": nbytes, "GB/s": gbs,
+                        "hbm_frac": gbs / peaks["hbm_gbs"], "tokens/s": T / (us * 1e-6)}
+    return out
 
 
 def reduce_max(v: float, device) -> float:

@@ -42,6 +42,25 @@ def layer_for(spec: W.LayerSpec, seed: int = 0, experts: bool = True):
     return layer
 
 
+def check_output(got: np.ndarray, ref: np.ndarray, tol: float, bf16_out: bool) -> float:
+    """Layer output check: |got - ref| <= tol * RMS(ref) + (output rounding) per element.
+
+    The output is stored in the activation dtype.  Rounding the exact fp64
+    result to bf16 moves an element by up to half an ulp, <= 2^-8 |ref|, which
+    on large-magnitude elements is already close to 2e-2 of the RMS (for the
+    GPT-OSS-120B-shaped layer: 1.75e-2 on the sampled tokens, 2^-8 x max|y|/RMS
+    = 2.3e-2 in the worst case), so that rounding is allowed on top of the bound.
+    Returns the raw max |got - ref| / RMS(ref) for the record.
+    """
+    rms = float(np.sqrt(np.mean(np.square(ref))))
+    allow = (2.0 ** -8 if bf16_out else 2.0 ** -23) * np.abs(ref)
+    excess = np.abs(got - ref) - (tol * rms + allow)
+    raw = float(np.max(np.abs(got - ref))) / max(rms, 1e-30)
+    assert np.all(excess <= 0), f"max excess {excess.max():.3e}; raw max err / RMS = {raw:.3e}"
+    print(f"max err / RMS = {raw:.3e}")
+    return raw
+
+
 def rel_rms(got: np.ndarray, ref: np.ndarray) -> float:
     rms = float(np.sqrt(np.mean(np.square(ref))))
     return float(np.max(np.abs(got - ref))) / max(rms, 1e-30)
