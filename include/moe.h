@@ -150,6 +150,29 @@ MOE_API moe_status_t moe_permute(const moe_config_t* cfg, int64_t T, const int32
                          int32_t* expert_off, int32_t* row_of_slot, int32_t* slot_of_row, void* x_perm, void* ws,
                          size_t ws_bytes, void* stream);
 
+/* moe_permute without a workspace argument and without any allocation.
+ * The pages have no counterpart: this entry point exists for callers that are
+ * not allowed to allocate device memory -- a plugin or custom operator inside a
+ * host framework or inference server whose allocator owns the whole GPU, or a
+ * service whose device-memory budget is fixed at start-up -- and so cannot call
+ * cudaMalloc for moe_permute's scratch or keep a workspace between calls.
+ * Same arguments, results and errors as moe_permute, except:
+ *  - the histogram/scan scratch is a fixed array inside the library (256 KiB,
+ *    one per GPU that loads the library, held until the process exits), so
+ *    num_local_experts * ceil(T / 256) must be at most 32768 (e.g. T <= 65536
+ *    with E = 128); larger sizes return MOE_ERR_UNSUPPORTED and launch nothing;
+ *  - the first call on a device looks up that array's device address (a
+ *    runtime call, no allocation); make that first call before any stream
+ *    capture;
+ *  - every call on a device shares the array and it keeps the last call's
+ *    contents (each call writes every word it reads, so nothing needs clearing),
+ *    hence calls that may overlap on the GPU (other streams, other threads) race
+ *    and must be serialised by the caller.
+ * It calls no cudaMalloc, cudaFree or other allocating routine. */
+MOE_API moe_status_t moe_permute_noalloc(const moe_config_t* cfg, int64_t T, const int32_t* topk_ids, const void* x,
+                                         int32_t* expert_off, int32_t* row_of_slot, int32_t* slot_of_row,
+                                         void* x_perm, void* stream);
+
 /* Per-expert FFN over the permuted rows (R = T*k):
  *   x_perm [R, D], expert_off [E+1] (as produced by moe_permute; read on the device)
  *   -> h [R, F]: clipped SwiGLU of the gate/up projections (+ biases),

@@ -56,6 +56,7 @@ SIGNATURES = {
     "moe_workspace_size": (ctypes.c_size_t, [_CFG, _I64]),
     "moe_router_topk": (_ST, [_CFG, _I64, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (_ST, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_permute_noalloc": (_ST, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_ffn": (_ST, [_CFG, _I64, _P, _P, _W, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_combine": (_ST, [_CFG, _I64, _P, _P, _P, _P, _P]),
     "moe_layer_forward": (_ST, [_CFG, _I64, _P, _P, _P, _W, _P, _P, _P, _P, ctypes.c_size_t, _P]),

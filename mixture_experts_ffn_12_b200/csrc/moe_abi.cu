@@ -176,6 +176,30 @@ moe_status_t run_experts(const moe_config_t* c, const Launch& L, int64_t T, cons
   return st;
 }
 
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: the dispatch with its scratch in a fixed device array
+// ---------------------------------------------------------------------------
+// Histogram and scan scratch of moe_permute_noalloc: 2 * E * ceil(T / 256)
+// int32 words at most kNoAllocWords (256 KiB).  One copy per GPU that loads
+// the library, kept until the process exits; every call on a device shares it.
+constexpr size_t kNoAllocWords = 65536;
+static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocWords];
+
+// Host code cannot use g_permute_scratch's name as a device address, so the
+// address is looked up once per device (with that device current) and cached.
+int32_t* permute_scratch_address(int dev) {
+  static std::mutex mu;
+  static int32_t* addr[64] = {};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> g(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int32_t*>(p);
+  }
+  return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -245,6 +269,30 @@ moe_status_t moe_permute(const moe_config_t* cfg, int64_t T, const int32_t* topk
   return cuda_status(moe::permute(L, cfg->dtype == MOE_BF16, T, cfg->hidden_size, cfg->num_local_experts,
                                   cfg->num_experts_per_tok, topk_ids, x, expert_off, row_of_slot, slot_of_row,
                                   x_perm, static_cast<int32_t*>(ws)));
+}
+
+moe_status_t moe_permute_noalloc(const moe_config_t* cfg, int64_t T, const int32_t* topk_ids, const void* x,
+                                 int32_t* expert_off, int32_t* row_of_slot, int32_t* slot_of_row, void* x_perm,
+                                 void* stream) {
+  moe_status_t s = check_cfg(cfg);
+  if (s != MOE_OK) return s;
+  if (!check_T(T, cfg->num_experts_per_tok)) return MOE_ERR_INVALID_ARG;
+  if (!ptr_ok(expert_off)) return MOE_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (!ptr_ok(topk_ids) || !ptr_ok(row_of_slot) || !ptr_ok(slot_of_row)) return MOE_ERR_INVALID_ARG;
+    if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+    if (x != nullptr && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+    if (moe::permute_scratch_words(T, cfg->num_local_experts) > kNoAllocWords) return MOE_ERR_UNSUPPORTED;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t* scratch = permute_scratch_address(dev);
+  if (scratch == nullptr) return MOE_ERR_CUDA;
+  Launch L;
+  if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
+  return cuda_status(moe::permute(L, cfg->dtype == MOE_BF16, T, cfg->hidden_size, cfg->num_local_experts,
+                                  cfg->num_experts_per_tok, topk_ids, x, expert_off, row_of_slot, slot_of_row,
+                                  x_perm, scratch));
 }
 
 moe_status_t moe_expert_ffn(const moe_config_t* cfg, int64_t T, const void* x_perm, const int32_t* expert_off,
