@@ -213,6 +213,14 @@ MOE_API moe_status_t moe_last_device_error(void);
  * this process until the next call of this function (n = 0 clears). */
 MOE_API void moe_set_stage_events(void* const* starts, void* const* stops, int32_t n);
 
+/* Tuning knob for the bf16 expert GEMMs of every later call in this process:
+ * 0 = choose by size (default: the weight-stationary decode kernel while the
+ * experts average at most 16 routed rows, single-CTA 128-row tiles otherwise),
+ * 1 = single-CTA tiles, 2 = CTA-pair tiles (256 rows), 3 = decode kernel.
+ * Results are the same up to fp32 accumulation order.  MOE_ERR_INVALID_ARG for
+ * other values. */
+MOE_API moe_status_t moe_set_expert_gemm_variant(int32_t variant);
+
 /* Number of kernels this library has launched in this process so far. */
 MOE_API uint64_t moe_launch_count(void);
 

@@ -64,6 +64,7 @@ SIGNATURES = {
     "moe_set_stage_events": (None, [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p),
                                     ctypes.c_int32]),
     "moe_launch_count": (ctypes.c_uint64, []),
+    "moe_set_expert_gemm_variant": (_ST, [ctypes.c_int32]),
     "moe_set_wait_limit_ns": (None, [ctypes.c_uint64]),
 }
 

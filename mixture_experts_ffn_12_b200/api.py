@@ -183,6 +183,11 @@ def last_device_error() -> int:
     return _lib.load().moe_last_device_error()
 
 
+def set_expert_gemm_variant(variant: int) -> None:
+    """0 = by size, 1 = single-CTA tiles, 2 = CTA-pair tiles (bf16 expert GEMMs)."""
+    _check(_lib.load().moe_set_expert_gemm_variant(variant), "moe_set_expert_gemm_variant")
+
+
 def set_wait_limit_ns(ns: int) -> None:
     _lib.load().moe_set_wait_limit_ns(ns)
 

@@ -12,6 +12,8 @@
 #include <mutex>
 
 #include "grouped_gemm.cuh"
+#include "decode_gemm.cuh"
+#include "grouped_gemm_pair.cuh"
 #include "internal.h"
 #include "simt_gemm.cuh"
 
@@ -76,6 +78,74 @@ static cudaError_t launch(const Launch& L, const CUtensorMap& a, const CUtensorM
   return cudaGetLastError();
 }
 
+// CTA-pair kernels (cluster of 2; grid = 2 x clusters).
+template <int TNH, int EPI, int STAGES>
+static cudaError_t launch_pair(const Launch& L, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                               const GemmArgs& args, int64_t max_tiles) {
+  if (max_tiles <= 0) return cudaSuccess;
+  auto kern = grouped_gemm_pair_kernel<TNH, EPI, STAGES>;
+  constexpr int smem = PairLayout<TNH>::smem_bytes(STAGES);
+  static_assert(smem <= 232448, "shared memory budget");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static std::mutex mu;
+  static uint64_t configured = 0;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (dev >= 64 || !((configured >> dev) & 1u)) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) configured |= uint64_t(1) << dev;
+    }
+  }
+  const int clusters = static_cast<int>(std::min<int64_t>(max_tiles, L.num_sms / 2));
+  kern<<<2 * clusters, kGemmThreads, smem, L.stream>>>(a, b0, b1, args);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// Expert-GEMM variant (moe_set_expert_gemm_variant): 0 = by size, 1 = single-CTA
+// tiles, 2 = CTA-pair tiles, 3 = weight-stationary decode kernel.
+inline std::atomic<int> g_gemm_variant{0};
+
+enum GemmKind { GK_SINGLE = 1, GK_PAIR = 2, GK_DECODE = 3 };
+
+// By default: the decode kernel while experts average at most 16 rows (the
+// layer is a weight stream), single-CTA 128-row tiles otherwise.
+static GemmKind gemm_kind(int64_t R, int E) {
+  const int v = g_gemm_variant.load();
+  if (v >= 1 && v <= 3) return static_cast<GemmKind>(v);
+  return R <= int64_t(16) * E ? GK_DECODE : GK_SINGLE;
+}
+static bool use_pair(int64_t R, int E) { return gemm_kind(R, E) == GK_PAIR; }
+
+constexpr int kDecTok = 32;
+
+template <int EPI>
+static cudaError_t launch_decode(const Launch& L, const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x,
+                                 const GemmArgs& args, int64_t max_units) {
+  if (max_units <= 0) return cudaSuccess;
+  auto kern = decode_gemm_kernel<EPI, kDecTok, kDecStages>;
+  constexpr int smem = DecLayout<kDecTok>::smem_bytes(kDecStages);
+  static_assert(smem <= 232448, "shared memory budget");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static std::mutex mu;
+  static uint64_t configured = 0;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (dev >= 64 || !((configured >> dev) & 1u)) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) configured |= uint64_t(1) << dev;
+    }
+  }
+  const int grid = static_cast<int>(std::min<int64_t>(max_units, L.num_sms));
+  kern<<<grid, kGemmThreads, smem, L.stream>>>(w0, w1, x, args);
+  count_launch();
+  return cudaGetLastError();
+}
+
 static GemmArgs base_args(const Launch& L) {
   GemmArgs a{};
   a.wait_limit_ns = L.wait_limit_ns;
@@ -86,6 +156,8 @@ static GemmArgs base_args(const Launch& L) {
 static int64_t max_row_blocks(int64_t R, int G) { return (R + kBM - 1) / kBM + G; }
 
 constexpr int kStages = 4;
+constexpr int kPairStages = 6;
+constexpr int kTNHalf = 120;     // pair tiles: each CTA holds 120 B rows (N = 240)
 constexpr int kTNGateUp = 120;   // 2 x 120 = 240 MMA columns, F = 2880 = 24 x 120
 constexpr int kTNDown = 240;     // D = 2880 = 12 x 240
 
@@ -107,7 +179,11 @@ cudaError_t router_tc(const Launch& L, int64_t T, int D, int E, int k, const voi
   a.topk_ids = ids;
   a.topk_wout = w;
   a.topk_k = k;
-  return launch<__nv_bfloat16, 256, 1, EPI_TOPK, kStages>(L, ta, tb, tb, a, (T + kBM - 1) / kBM);
+  // one CTA per 128 tokens: few CTAs stream x, so the ring is as deep as shared memory allows
+  const int64_t tiles = (T + kBM - 1) / kBM;
+  if (mma_n <= 64) return launch<__nv_bfloat16, 64, 1, EPI_TOPK, 9>(L, ta, tb, tb, a, tiles);
+  if (mma_n <= 128) return launch<__nv_bfloat16, 128, 1, EPI_TOPK, 6>(L, ta, tb, tb, a, tiles);
+  return launch<__nv_bfloat16, 256, 1, EPI_TOPK, kStages>(L, ta, tb, tb, a, tiles);
 }
 
 cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,
@@ -149,6 +225,18 @@ cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, i
   a.alpha = alpha;
   a.out = h;
   a.ldo = F;
+  if (gemm_kind(R, E) == GK_DECODE) {
+    CUtensorMap wg, wu, tx;
+    if ((e = make_tmap(&wg, w.w_gate, false, D, F, E, 64)) != cudaSuccess) return e;
+    if ((e = make_tmap(&wu, w.w_up, false, D, F, E, 64)) != cudaSuccess) return e;
+    if ((e = make_tmap(&tx, x_perm, false, D, R, 0, kDecTok)) != cudaSuccess) return e;
+    const int64_t units = (std::min<int64_t>(E, R) + R / kDecTok) * ((F + 63) / 64);
+    return launch_decode<EPI_SWIGLU>(L, wg, wu, tx, a, units);
+  }
+  if (use_pair(R, E)) {
+    const int64_t ptiles = ((R + kPairBM - 1) / kPairBM + E) * ((F + kTNHalf - 1) / kTNHalf);
+    return launch_pair<kTNHalf, EPI_SWIGLU, kPairStages>(L, ta, tg, tu, a, ptiles);
+  }
   const int64_t tiles = max_row_blocks(R, E) * ((F + kTNGateUp - 1) / kTNGateUp);
   return launch<__nv_bfloat16, kTNGateUp, 2, EPI_SWIGLU, kStages>(L, ta, tg, tu, a, tiles);
 }
@@ -182,7 +270,6 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
   CUtensorMap ta, tb;
   cudaError_t e;
   if ((e = make_tmap(&ta, h, !bf16, F, R, 0, kBM)) != cudaSuccess) return e;
-  if ((e = make_tmap(&tb, w.w_down, !bf16, F, D, E, kTNDown)) != cudaSuccess) return e;
   GemmArgs a = base_args(L);
   a.group_off = expert_off;
   a.num_groups = E;
@@ -194,6 +281,22 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
   a.ldo = D;
   a.slot_of_row = slot_of_row;
   a.topk_w = topk_w;
+  if (gemm_kind(R, E) == GK_DECODE) {
+    CUtensorMap wd, th;
+    if ((e = make_tmap(&wd, w.w_down, false, F, D, E, 128)) != cudaSuccess) return e;
+    if ((e = make_tmap(&th, h, false, F, R, 0, kDecTok)) != cudaSuccess) return e;
+    const int64_t units = (std::min<int64_t>(E, R) + R / kDecTok) * ((D + 127) / 128);
+    if (slot_of_row != nullptr) return launch_decode<EPI_BIAS_WSCATTER>(L, wd, wd, th, a, units);
+    return launch_decode<EPI_BIAS>(L, wd, wd, th, a, units);
+  }
+  const bool pair = use_pair(R, E);
+  if ((e = make_tmap(&tb, w.w_down, !bf16, F, D, E, pair ? kTNHalf : kTNDown)) != cudaSuccess) return e;
+  if (pair) {
+    const int64_t ptiles = ((R + kPairBM - 1) / kPairBM + E) * ((D + 2 * kTNHalf - 1) / (2 * kTNHalf));
+    if (slot_of_row != nullptr)
+      return launch_pair<kTNHalf, EPI_BIAS_WSCATTER, kPairStages>(L, ta, tb, tb, a, ptiles);
+    return launch_pair<kTNHalf, EPI_BIAS, kPairStages>(L, ta, tb, tb, a, ptiles);
+  }
   const int64_t tiles = max_row_blocks(R, E) * ((D + kTNDown - 1) / kTNDown);
   if (slot_of_row != nullptr)
     return launch<__nv_bfloat16, kTNDown, 1, EPI_BIAS_WSCATTER, kStages>(L, ta, tb, tb, a, tiles);

@@ -387,6 +387,12 @@ void moe_set_stage_events(void* const* starts, void* const* stops, int32_t n) {
 
 uint64_t moe_launch_count(void) { return moe::g_launches.load(); }
 
+moe_status_t moe_set_expert_gemm_variant(int32_t variant) {
+  if (variant < 0 || variant > 3) return MOE_ERR_INVALID_ARG;
+  moe::g_gemm_variant.store(variant);
+  return MOE_OK;
+}
+
 void moe_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns == 0 ? 1000000000ull : ns); }
 
 }  // extern "C"

@@ -38,6 +38,7 @@ __device__ __forceinline__ float dot_row16(const T* a, const T* b, int D, int la
   const uint4* pa = reinterpret_cast<const uint4*>(a);
   const uint4* pb = reinterpret_cast<const uint4*>(b);
   float acc = 0.0f;
+#pragma unroll 4
   for (int c = lane; c < nchunk; c += 32) {
     const uint4 ua = pa[c], ub = pb[c];
     if constexpr (sizeof(T) == 4) {
@@ -276,6 +277,81 @@ __global__ void permute_gather_kernel(const uint4* __restrict__ x, const int32_t
   }
 }
 
+// The whole dispatch of at most one chunk (T <= 256) in one CTA: lane masks, the
+// per-expert scan, ranks, both index maps, and the row copies (decode sizes).
+constexpr int kSmallMaxRows = kChunk * 8;   // T <= 256 tokens, k <= 8
+constexpr int kSmallCopyRows = 32;          // above this many rows the copy runs on many CTAs
+__global__ void __launch_bounds__(kChunk) permute_small_kernel(const int32_t* __restrict__ ids, int T, int k, int E,
+                                                               const uint4* __restrict__ x, int vec_per_row,
+                                                               int32_t* __restrict__ expert_off,
+                                                               int32_t* __restrict__ row_of_slot,
+                                                               int32_t* __restrict__ slot_of_row,
+                                                               uint4* __restrict__ x_perm) {
+  __shared__ uint32_t mask[kChunkWarps][256];
+  __shared__ int base[257];
+  __shared__ int sor[kSmallMaxRows];
+  build_masks(mask, ids, T, k, E);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) {
+    // exclusive scan of the per-expert counts, 8 experts per lane
+    int c[8], tot = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      int v = 0;
+      if (e < E) {
+#pragma unroll
+        for (int w = 0; w < kChunkWarps; ++w) v += __popc(mask[w][e]);
+      }
+      c[i] = v;
+      tot += v;
+    }
+    int incl = tot;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += o;
+    }
+    int run = incl - tot;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      if (e < E) base[e] = run;
+      run += c[i];
+    }
+    if (lane == 31) base[E] = incl;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) expert_off[e] = base[e];
+  const int R = T * k;
+  const int t = threadIdx.x;
+  if (t < T) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[t * k + j];
+      if (e < 0 || e >= E) continue;
+      int r = base[e] + __popc(mask[warp][e] & lt);
+      for (int w = 0; w < warp; ++w) r += __popc(mask[w][e]);
+      if (r < 0 || r >= R) {
+        flag_error(DEVERR_BOUNDS);
+        continue;
+      }
+      row_of_slot[t * k + j] = r;
+      slot_of_row[r] = t * k + j;
+      sor[r] = t * k + j;
+    }
+  }
+  __syncthreads();
+  if (x == nullptr) return;
+  for (int r = warp; r < R; r += kChunkWarps) {
+    const int src = sor[r] / k;
+    if (src < 0 || src >= T) continue;
+    const uint4* a = x + static_cast<size_t>(src) * vec_per_row;
+    uint4* b = x_perm + static_cast<size_t>(r) * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) b[v] = a[v];
+  }
+}
+
 cudaError_t permute(const Launch& L, bool bf16, int64_t T, int D, int E, int k, const int32_t* ids, const void* x,
                     int32_t* expert_off, int32_t* row_of_slot, int32_t* slot_of_row, void* x_perm,
                     int32_t* scratch) {
@@ -283,13 +359,25 @@ cudaError_t permute(const Launch& L, bool bf16, int64_t T, int D, int E, int k, 
     return cudaMemsetAsync(expert_off, 0, sizeof(int32_t) * (E + 1), L.stream);
   }
   const int nchunks = static_cast<int>((T + kChunk - 1) / kChunk);
-  int32_t* cnt = scratch;
-  int32_t* base = scratch + static_cast<size_t>(nchunks) * E;
-  permute_count_kernel<<<nchunks, kChunk, 0, L.stream>>>(ids, static_cast<int>(T), k, E, nchunks, cnt);
-  permute_scan_kernel<<<1, 1024, 0, L.stream>>>(cnt, nchunks * E, E, nchunks, base, expert_off);
-  permute_scatter_kernel<<<nchunks, kChunk, 0, L.stream>>>(ids, static_cast<int>(T), k, E, nchunks, base,
-                                                           row_of_slot, slot_of_row);
-  count_launch(3);
+  if (nchunks == 1) {
+    // one CTA builds the maps; it also copies the rows when there are few of them
+    const bool rows = x != nullptr && x_perm != nullptr;
+    const bool copy_here = rows && T * k <= kSmallCopyRows;
+    permute_small_kernel<<<1, kChunk, 0, L.stream>>>(ids, static_cast<int>(T), k, E,
+                                                     copy_here ? static_cast<const uint4*>(x) : nullptr,
+                                                     D * (bf16 ? 2 : 4) / 16, expert_off, row_of_slot, slot_of_row,
+                                                     copy_here ? static_cast<uint4*>(x_perm) : nullptr);
+    count_launch();
+    if (!rows || copy_here) return cudaGetLastError();
+  } else {
+    int32_t* cnt = scratch;
+    int32_t* base = scratch + static_cast<size_t>(nchunks) * E;
+    permute_count_kernel<<<nchunks, kChunk, 0, L.stream>>>(ids, static_cast<int>(T), k, E, nchunks, cnt);
+    permute_scan_kernel<<<1, 1024, 0, L.stream>>>(cnt, nchunks * E, E, nchunks, base, expert_off);
+    permute_scatter_kernel<<<nchunks, kChunk, 0, L.stream>>>(ids, static_cast<int>(T), k, E, nchunks, base,
+                                                             row_of_slot, slot_of_row);
+    count_launch(3);
+  }
   if (x != nullptr && x_perm != nullptr) {
     const int R = static_cast<int>(T * k);
     const int vpr = D * (bf16 ? 2 : 4) / 16;

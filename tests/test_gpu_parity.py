@@ -35,7 +35,11 @@ WIDE_K = W.tiny_spec(T=260, D=64, E=16, k=8, F=48, dtype="bf16", cfg_id=203)
 ONE_EXPERT = W.tiny_spec(T=40, D=32, E=1, k=1, F=32, dtype="bf16", cfg_id=204)
 MXFP4_SMALL = W.tiny_spec(T=280, D=128, E=6, k=2, F=160, dtype="bf16", wfmt="mxfp4", cfg_id=205)
 
-SMALL_SPECS = [W.TINY_FP32, RAGGED_BF16, RAGGED_F32, WIDE_K, ONE_EXPERT, MXFP4_SMALL]
+# >= 128 rows per expert on average: runs the CTA-pair kernels; ragged F and D tiles, an expert with no rows
+PAIR_RAGGED = W.tiny_spec(T=900, D=256, E=5, k=2, F=272, dtype="bf16", cfg_id=206, dead_experts=(3,),
+                          router_w_std=0.2)
+
+SMALL_SPECS = [W.TINY_FP32, RAGGED_BF16, RAGGED_F32, WIDE_K, ONE_EXPERT, MXFP4_SMALL, PAIR_RAGGED]
 DECODE_SPECS = [W.gptoss20b_decode(t) for t in W.GPTOSS20B_DECODE_T]
 
 
@@ -227,3 +231,20 @@ def test_layer_forward_repeatable(api):
     y2 = api.layer_forward(cfg, d["x"], d["w_router"], d["b_router"], ew)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("variant", [1, 2, 3], ids=["single_cta", "cta_pair", "decode"])
+@pytest.mark.parametrize("spec", [RAGGED_BF16, PAIR_RAGGED, W.gptoss20b_decode(8)], ids=lambda s: s.name)
+def test_layer_forward_each_gemm_variant(api, spec, variant):
+    """Every bf16 expert-GEMM kernel on the same layer: single-CTA 128-row tiles, CTA pairs
+    (256 rows), and the weight-stationary decode kernel (token chunks of 32, so experts with
+    more rows run several chunks)."""
+    layer = layer_for(spec)
+    api.set_expert_gemm_variant(variant)
+    try:
+        y, gid, _ = _run_layer(api, spec, layer)
+    finally:
+        api.set_expert_gemm_variant(0)
+    ref = O.layer_tokens(layer, np.arange(spec.T), spec.k, spec.limit, spec.alpha)
+    check_ids(gid, ref["ids"], ref["logits"])
+    check_output(f64(y), ref["y"], tol_for(spec), True)

@@ -55,6 +55,7 @@ class LayerSpec:
     zipf_s: float = 1.1
     expert_w_std: Optional[float] = None   # None -> 1/sqrt(fan_in)
     expert_b_std: float = 0.01
+    dead_experts: tuple = ()               # router bias -30 for these: they receive no tokens
     cfg_id: int = 0                        # seeds the streams; distinct per recipe
 
     @property
@@ -164,6 +165,8 @@ def make_layer(spec: LayerSpec, seed: int = 0,
         br = zipf_log_bias(E, spec.zipf_s).astype(np.float32)
     else:
         br = np.zeros(E, dtype=np.float32)
+    for e in spec.dead_experts:
+        br[e] = -30.0
     out["b_router"] = f32_to_bf16_bits(br) if spec.dtype == "bf16" else br.astype(np.float32)
 
     if with_experts:
