@@ -208,3 +208,21 @@ class MoELayer:
     def __call__(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, topk_ids=None, topk_w=None) -> torch.Tensor:
         return layer_forward(self.cfg, x, self.w_router, self.b_router, self.experts, y=y,
                              ws=self.workspace(x.shape[0]), topk_ids=topk_ids, topk_w=topk_w)
+
+    def graphed(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, topk_ids=None, topk_w=None):
+        """Capture one forward on these fixed buffers into a CUDA graph; returns (replay, y).
+
+        The library makes no host synchronisation and allocates nothing, so its
+        launches are captured as they are; ``replay()`` re-runs them on whatever
+        ``x`` holds at that time.  Removes host launch overhead (decode sizes).
+        """
+        if y is None:
+            y = torch.empty((x.shape[0], self.cfg.hidden_size), dtype=x.dtype, device=x.device)
+        ws = self.workspace(x.shape[0])
+        self(x, y=y, topk_ids=topk_ids, topk_w=topk_w)          # warm: per-device set-up outside capture
+        torch.cuda.synchronize(x.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            layer_forward(self.cfg, x, self.w_router, self.b_router, self.experts, y=y, ws=ws,
+                          topk_ids=topk_ids, topk_w=topk_w)
+        return g.replay, y

@@ -28,7 +28,7 @@ namespace moe {
 // ---------------------------------------------------------------------------
 // router, SIMT: one block (16 warps) per token
 // ---------------------------------------------------------------------------
-constexpr int kRouterWarps = 16;
+constexpr int kRouterWarps = 32;   // one block per token: a warp per expert for E <= 32
 
 template <typename T>
 __device__ __forceinline__ float dot_row16(const T* a, const T* b, int D, int lane) {
@@ -38,7 +38,7 @@ __device__ __forceinline__ float dot_row16(const T* a, const T* b, int D, int la
   const uint4* pa = reinterpret_cast<const uint4*>(a);
   const uint4* pb = reinterpret_cast<const uint4*>(b);
   float acc = 0.0f;
-#pragma unroll 4
+#pragma unroll 6
   for (int c = lane; c < nchunk; c += 32) {
     const uint4 ua = pa[c], ub = pb[c];
     if constexpr (sizeof(T) == 4) {

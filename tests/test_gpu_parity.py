@@ -248,3 +248,20 @@ def test_layer_forward_each_gemm_variant(api, spec, variant):
     ref = O.layer_tokens(layer, np.arange(spec.T), spec.k, spec.limit, spec.alpha)
     check_ids(gid, ref["ids"], ref["logits"])
     check_output(f64(y), ref["y"], tol_for(spec), True)
+
+
+def test_cuda_graph_replay_matches_eager(api):
+    """A captured forward replays the same kernels on new contents of the input buffer."""
+    spec = W.gptoss20b_decode(8)
+    layer = layer_for(spec)
+    d = dev(layer, api)
+    moe = api.MoELayer(api.config_from_spec(spec), d["w_router"], d["b_router"], api.expert_weights_from(d))
+    x = d["x"].clone()
+    replay, y_graph = moe.graphed(x)
+    x2 = torch.roll(d["x"], shifts=3, dims=0).contiguous()
+    x.copy_(x2)
+    replay()
+    y_eager = moe(x2)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    assert torch.equal(y_graph, y_eager)
