@@ -117,8 +117,9 @@ MOE_API moe_status_t moe_config_check(const moe_config_t* cfg);
  * scratch).  0 when T == 0; (size_t)-1 if cfg is invalid. */
 MOE_API size_t moe_permute_workspace_size(const moe_config_t* cfg, int64_t T);
 
-/* Bytes of workspace moe_expert_ffn needs (0 for dense weights; MXFP4 needs room
- * for dequantised expert weights). (size_t)-1 if cfg is invalid. */
+/* Bytes of workspace moe_expert_ffn needs: 0 for every supported configuration
+ * (MXFP4 weights are dequantised inside the GEMM mainloop); kept so callers can
+ * size a workspace without knowing that.  (size_t)-1 if cfg is invalid. */
 MOE_API size_t moe_expert_ffn_workspace_size(const moe_config_t* cfg, int64_t T);
 
 /* Bytes of workspace moe_layer_forward needs for T tokens: routing ids and
@@ -177,9 +178,10 @@ MOE_API moe_status_t moe_permute_noalloc(const moe_config_t* cfg, int64_t T, con
  *   x_perm [R, D], expert_off [E+1] (as produced by moe_permute; read on the device)
  *   -> h [R, F]: clipped SwiGLU of the gate/up projections (+ biases),
  *      y_perm [R, D]: h Wd[e]^T + bd[e] for the expert e that owns each row.
- * Computed on the tcgen05 tensor cores with fp32 accumulation (bf16 operands;
- * fp32 layers use TF32 operands).  ws: moe_expert_ffn_workspace_size bytes
- * (may be NULL when that is 0). */
+ * Computed on the tcgen05 tensor cores with fp32 accumulation from bf16
+ * operands (MXFP4 weights are decoded to bf16 in shared memory inside the GEMM
+ * mainloop; fp32 layers run in fp32 FMA).  ws: moe_expert_ffn_workspace_size
+ * bytes (may be NULL when that is 0). */
 MOE_API moe_status_t moe_expert_ffn(const moe_config_t* cfg, int64_t T, const void* x_perm, const int32_t* expert_off,
                             const moe_expert_weights_t* weights, void* h, void* y_perm, void* ws, size_t ws_bytes,
                             void* stream);

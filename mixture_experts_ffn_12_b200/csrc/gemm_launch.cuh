@@ -14,6 +14,7 @@
 #include "grouped_gemm.cuh"
 #include "decode_gemm.cuh"
 #include "grouped_gemm_pair.cuh"
+#include "grouped_gemm_pair_mx.cuh"
 #include "internal.h"
 #include "simt_gemm.cuh"
 
@@ -49,6 +50,21 @@ static cudaError_t make_tmap(CUtensorMap* m, const void* ptr, bool f32, uint64_t
   const CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                         groups ? 3 : 2, const_cast<void*>(ptr), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Packed MXFP4 rows: [groups, rows, K/2] bytes, boxes of box_rows x 32 bytes (64 codes), no swizzle.
+static cudaError_t make_tmap_packed(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows, uint64_t groups,
+                                   uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {K / 2, rows, groups};
+  const cuuint64_t strides[2] = {K / 2, (K / 2) * rows};
+  const cuuint32_t box[3] = {32, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -100,6 +116,31 @@ static cudaError_t launch_pair(const Launch& L, const CUtensorMap& a, const CUte
   }
   const int clusters = static_cast<int>(std::min<int64_t>(max_tiles, L.num_sms / 2));
   kern<<<2 * clusters, kGemmThreads, smem, L.stream>>>(a, b0, b1, args);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <int TNH, int EPI, int STAGES>
+static cudaError_t launch_pair_mx(const Launch& L, const CUtensorMap& a, const CUtensorMap& p0, const CUtensorMap& p1,
+                                  const GemmArgs& args, int64_t max_tiles) {
+  if (max_tiles <= 0) return cudaSuccess;
+  auto kern = grouped_gemm_pair_mx_kernel<TNH, EPI, STAGES>;
+  constexpr int smem = PairMxLayout<TNH>::smem_bytes(STAGES);
+  static_assert(smem <= 232448, "shared memory budget");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static std::mutex mu;
+  static uint64_t configured = 0;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (dev >= 64 || !((configured >> dev) & 1u)) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) configured |= uint64_t(1) << dev;
+    }
+  }
+  const int clusters = static_cast<int>(std::min<int64_t>(max_tiles, L.num_sms / 2));
+  kern<<<2 * clusters, kMxThreads, smem, L.stream>>>(a, p0, p1, args);
   count_launch();
   return cudaGetLastError();
 }
@@ -184,6 +225,61 @@ cudaError_t router_tc(const Launch& L, int64_t T, int D, int E, int k, const voi
   if (mma_n <= 64) return launch<__nv_bfloat16, 64, 1, EPI_TOPK, 9>(L, ta, tb, tb, a, tiles);
   if (mma_n <= 128) return launch<__nv_bfloat16, 128, 1, EPI_TOPK, 6>(L, ta, tb, tb, a, tiles);
   return launch<__nv_bfloat16, 256, 1, EPI_TOPK, kStages>(L, ta, tb, tb, a, tiles);
+}
+
+constexpr int kMxStages = 5;
+
+cudaError_t expert_gateup_mxfp4(const Launch& L, int64_t R, int D, int F, int E, const void* x_perm,
+                                const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h) {
+  if (R == 0) return cudaSuccess;
+  CUtensorMap ta, pg, pu;
+  cudaError_t e;
+  if ((e = make_tmap(&ta, x_perm, false, D, R, 0, kBM)) != cudaSuccess) return e;
+  if ((e = make_tmap_packed(&pg, w.w_gate, D, F, E, kTNHalf)) != cudaSuccess) return e;
+  if ((e = make_tmap_packed(&pu, w.w_up, D, F, E, kTNHalf)) != cudaSuccess) return e;
+  GemmArgs a = base_args(L);
+  a.group_off = expert_off;
+  a.num_groups = E;
+  a.m_total = static_cast<int>(R);
+  a.n_out = F;
+  a.k_dim = D;
+  a.bias0 = w.b_gate;
+  a.bias1 = w.b_up;
+  a.limit = limit;
+  a.alpha = alpha;
+  a.out = h;
+  a.ldo = F;
+  a.scale0 = w.s_gate;
+  a.scale1 = w.s_up;
+  const int64_t ptiles = ((R + kPairBM - 1) / kPairBM + E) * ((F + kTNHalf - 1) / kTNHalf);
+  return launch_pair_mx<kTNHalf, EPI_SWIGLU, kMxStages>(L, ta, pg, pu, a, ptiles);
+}
+
+cudaError_t expert_down_mxfp4(const Launch& L, int64_t R, int D, int F, int E, const void* h,
+                              const int32_t* expert_off, const ExpertWeights& w, const int32_t* slot_of_row,
+                              const float* topk_w, void* out) {
+  if (R == 0) return cudaSuccess;
+  CUtensorMap ta, pd;
+  cudaError_t e;
+  if ((e = make_tmap(&ta, h, false, F, R, 0, kBM)) != cudaSuccess) return e;
+  if ((e = make_tmap_packed(&pd, w.w_down, F, D, E, kTNHalf)) != cudaSuccess) return e;
+  GemmArgs a = base_args(L);
+  a.group_off = expert_off;
+  a.num_groups = E;
+  a.m_total = static_cast<int>(R);
+  a.n_out = D;
+  a.k_dim = F;
+  a.bias0 = w.b_down;
+  a.out = out;
+  a.ldo = D;
+  a.slot_of_row = slot_of_row;
+  a.topk_w = topk_w;
+  a.scale0 = w.s_down;
+  a.scale1 = w.s_down;
+  const int64_t ptiles = ((R + kPairBM - 1) / kPairBM + E) * ((D + 2 * kTNHalf - 1) / (2 * kTNHalf));
+  if (slot_of_row != nullptr)
+    return launch_pair_mx<kTNHalf, EPI_BIAS_WSCATTER, kMxStages>(L, ta, pd, pd, a, ptiles);
+  return launch_pair_mx<kTNHalf, EPI_BIAS, kMxStages>(L, ta, pd, pd, a, ptiles);
 }
 
 cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,

@@ -63,6 +63,8 @@ struct GemmArgs {
   float* topk_wout;            // EPI_TOPK [m_total, topk_k]
   int topk_k;
   unsigned long long wait_limit_ns;
+  const uint8_t* scale0;       // MXFP4: E8M0 scales of B0 / B1, [G, n_out, k_dim / 32]
+  const uint8_t* scale1;
 };
 
 constexpr int kBM = 128;           // rows per tile (MMA M)

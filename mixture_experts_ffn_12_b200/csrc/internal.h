@@ -55,8 +55,12 @@ cudaError_t combine_gather(const Launch& L, bool bf16, int64_t T, int D, int k, 
 // y[t] = sum_j ys[t*k + j]   (ys fp32, y dtype)
 cudaError_t combine_slots(const Launch& L, bool bf16, int64_t T, int D, int k, const void* ys, void* y);
 
-// MXFP4 -> bf16 weights ([rows, K/2] packed + [rows, K/32] scales -> [rows, K]).
-cudaError_t mxfp4_dequant(const Launch& L, int64_t rows, int K, const uint8_t* q, const uint8_t* s, void* out);
+// The same two projections with MXFP4 expert weights, dequantised inside the GEMM mainloop.
+cudaError_t expert_gateup_mxfp4(const Launch& L, int64_t R, int D, int F, int E, const void* x_perm,
+                                const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h);
+cudaError_t expert_down_mxfp4(const Launch& L, int64_t R, int D, int F, int E, const void* h,
+                              const int32_t* expert_off, const ExpertWeights& w, const int32_t* slot_of_row,
+                              const float* topk_w, void* out);
 
 cudaError_t read_and_clear_device_error(int* bits);
 

@@ -57,11 +57,8 @@ bool check_T(int64_t T, int k) { return T >= 0 && T * k < (int64_t(1) << 31); }
 
 size_t elem_size(const moe_config_t* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
 
-size_t ffn_ws_bytes(const moe_config_t* c, int64_t T) {
-  if (c->wfmt != MOE_W_MXFP4 || T == 0) return 0;
-  // dequantised gate and up weights (the down weights reuse the same space)
-  return 2 * align256(size_t(c->num_local_experts) * c->intermediate_size * c->hidden_size * 2);
-}
+// The expert GEMMs need no scratch (MXFP4 weights are dequantised in the mainloop).
+size_t ffn_ws_bytes(const moe_config_t*, int64_t) { return 0; }
 
 struct Layout {
   size_t ids, w, off, ros, sor, pscr, xperm, h, ys, ffn, total;
@@ -146,24 +143,12 @@ moe_status_t run_experts(const moe_config_t* c, const Launch& L, int64_t T, cons
   moe::ExpertWeights w = to_internal(wts);
   stage_mark(ST_GATEUP, true, L.stream);
   if (c->wfmt == MOE_W_MXFP4) {
-    uint8_t* buf = static_cast<uint8_t*>(ffn_ws);
-    void* wg = buf;
-    void* wu = buf + align256(size_t(E) * F * D * 2);
-    if (moe::mxfp4_dequant(L, int64_t(E) * F, D, static_cast<const uint8_t*>(wts->w_gate), wts->s_gate, wg) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    if (moe::mxfp4_dequant(L, int64_t(E) * F, D, static_cast<const uint8_t*>(wts->w_up), wts->s_up, wu) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    w.w_gate = wg;
-    w.w_up = wu;
-    if (moe::expert_gateup(L, true, R, D, F, E, x_perm, eoff, w, c->swiglu_limit, c->swiglu_alpha, h) != cudaSuccess)
+    if (moe::expert_gateup_mxfp4(L, R, D, F, E, x_perm, eoff, w, c->swiglu_limit, c->swiglu_alpha, h) !=
+        cudaSuccess)
       return MOE_ERR_CUDA;
     stage_mark(ST_GATEUP, false, L.stream);
     stage_mark(ST_DOWN, true, L.stream);
-    void* wd = buf;   // gate/up weights are dead once the gate/up kernel (stream-ordered) is done
-    if (moe::mxfp4_dequant(L, int64_t(E) * D, F, static_cast<const uint8_t*>(wts->w_down), wts->s_down, wd) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    w.w_down = wd;
-    const moe_status_t st = cuda_status(moe::expert_down(L, true, R, D, F, E, h, eoff, w, slot_of_row, topk_w, out));
+    const moe_status_t st = cuda_status(moe::expert_down_mxfp4(L, R, D, F, E, h, eoff, w, slot_of_row, topk_w, out));
     stage_mark(ST_DOWN, false, L.stream);
     return st;
   }

@@ -472,38 +472,6 @@ cudaError_t combine_slots(const Launch& L, bool bf16, int64_t T, int D, int k, c
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------------------
-// MXFP4 -> bf16 (E2M1 code: sign bit 3, exponent bits 2..1 with bias 1, mantissa bit 0;
-// E8M0 scale 2^(s-127) per 32 elements; element 2i = low nibble of byte i)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ float e2m1_to_float(uint32_t c) {
-  const uint32_t ex = (c >> 1) & 3u, man = c & 1u;
-  const float mag = ex == 0 ? 0.5f * static_cast<float>(man) : ldexpf(1.0f + 0.5f * static_cast<float>(man), ex - 1);
-  return (c & 8u) ? -mag : mag;
-}
-
-__global__ void mxfp4_dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ s, int64_t rows, int K,
-                                     __nv_bfloat16* __restrict__ out) {
-  const int64_t total = rows * (K / 2);
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / (K / 2);
-    const int b = static_cast<int>(i - r * (K / 2));
-    const uint32_t byte = q[i];
-    const float sc = ldexpf(1.0f, static_cast<int>(s[r * (K / 32) + (2 * b) / 32]) - 127);
-    out[r * K + 2 * b] = __float2bfloat16_rn(e2m1_to_float(byte & 0xFu) * sc);
-    out[r * K + 2 * b + 1] = __float2bfloat16_rn(e2m1_to_float(byte >> 4) * sc);
-  }
-}
-
-cudaError_t mxfp4_dequant(const Launch& L, int64_t rows, int K, const uint8_t* q, const uint8_t* s, void* out) {
-  if (rows == 0) return cudaSuccess;
-  const int blocks = elementwise_blocks(L, rows * (K / 2));
-  mxfp4_dequant_kernel<<<blocks, 256, 0, L.stream>>>(q, s, rows, K, static_cast<__nv_bfloat16*>(out));
-  count_launch();
-  return cudaGetLastError();
-}
-
 cudaError_t read_and_clear_device_error(int* bits) {
   int v = 0;
   cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));

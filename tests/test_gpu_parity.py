@@ -265,3 +265,25 @@ def test_cuda_graph_replay_matches_eager(api):
     torch.cuda.synchronize()
     assert api.last_device_error() == 0
     assert torch.equal(y_graph, y_eager)
+
+
+def test_mxfp4_matches_bf16_path_on_dequantised_weights(api):
+    """Every dequantised MXFP4 weight is a bf16 number, so the in-mainloop dequant must give the
+    bf16 CTA-pair kernel's result on those weights, bit for bit (same tiles, same accumulation order)."""
+    spec = MXFP4_SMALL
+    layer = layer_for(spec)
+    dense = dict(layer)
+    for name in ("gate", "up", "down"):
+        wq = O.mxfp4_dequant(layer[f"w_{name}"], layer[f"s_{name}"])
+        dense[f"w_{name}"] = W.f32_to_bf16_bits(wq.astype(np.float32))
+        dense.pop(f"s_{name}")
+        assert np.array_equal(W.bf16_bits_to_f32(dense[f"w_{name}"]).astype(np.float64), wq)
+    import dataclasses
+    y_mx, ids_mx, _ = _run_layer(api, spec, layer)
+    api.set_expert_gemm_variant(2)
+    try:
+        y_bf, ids_bf, _ = _run_layer(api, dataclasses.replace(spec, wfmt="dense"), dense)
+    finally:
+        api.set_expert_gemm_variant(0)
+    assert np.array_equal(ids_mx, ids_bf)
+    assert torch.equal(y_mx, y_bf)
