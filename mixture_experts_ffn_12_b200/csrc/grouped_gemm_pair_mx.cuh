@@ -227,7 +227,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag, lim)) { ok = false; break; }
-          if (!mbar_wait_cluster(&conv[s], ph, abort_flag, lim)) { ok = false; break; }
+          if (!mbar_wait(&conv[s], ph, abort_flag, lim)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * LY::STAGE_BYTES);
           const uint32_t b_addr = a_addr + LY::A_BYTES;
@@ -305,14 +305,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         uint8_t sc[(TNH + 15) / 16];
 #pragma unroll
         for (int j = 0; j < (TNH + 15) / 16; ++j) sc[j] = sc_next[j];
-        if (kb + 1 < KB) {
-#pragma unroll
-          for (int j = 0; j < (TNH + 15) / 16; ++j) {
-            const int r = r0 + 16 * j;
-            sc_next[j] = (r < TNH && b_row + r < args.n_out) ? srow[static_cast<size_t>(r) * KS + (kb + 1) * 2]
-                                                             : uint8_t(127);
-          }
-        }
         if (!__all_sync(0xffffffffu, mbar_wait(&pk[s], ph, abort_flag, lim))) { ok = false; break; }
         const uint8_t* sp = smem + s * LY::STAGE_BYTES + LY::A_BYTES + LY::B_BYTES;
         uint8_t* sb = smem + s * LY::STAGE_BYTES + LY::A_BYTES;
@@ -328,6 +320,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         fence_proxy_async_smem();     // generic-proxy stores -> visible to the tensor core
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(conv_leader + static_cast<uint32_t>(s) * 8u);
+        // next k-block's scales: issued after the fence so that it never waits for them
+        if (kb + 1 < KB) {
+#pragma unroll
+          for (int j = 0; j < (TNH + 15) / 16; ++j) {
+            const int r = r0 + 16 * j;
+            sc_next[j] = (r < TNH && b_row + r < args.n_out) ? srow[static_cast<size_t>(r) * KS + (kb + 1) * 2]
+                                                             : uint8_t(127);
+          }
+        }
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
     }
