@@ -227,6 +227,30 @@ cudaError_t router_tc(const Launch& L, int64_t T, int D, int E, int k, const voi
   return launch<__nv_bfloat16, 256, 1, EPI_TOPK, kStages>(L, ta, tb, tb, a, tiles);
 }
 
+// Router with K split over `splits` ranges: tile (m, s) writes fp32 partial logits of
+// tokens m*128.. over K range s to partial[s][T][E]; the top-k kernel sums them.
+cudaError_t router_tc_partial(const Launch& L, int64_t T, int D, int E, int splits, const void* x,
+                              const void* w_router, float* partial) {
+  const int mma_n = (E + 15) / 16 * 16;
+  CUtensorMap ta, tb;
+  cudaError_t e;
+  if ((e = make_tmap(&ta, x, false, D, T, 0, kBM)) != cudaSuccess) return e;
+  if ((e = make_tmap(&tb, w_router, false, D, E, 1, mma_n)) != cudaSuccess) return e;
+  GemmArgs a = base_args(L);
+  a.group_off = nullptr;
+  a.num_groups = 1;
+  a.m_total = static_cast<int>(T);
+  a.n_out = E;
+  a.k_dim = D;
+  a.mma_n = mma_n;
+  a.k_splits = splits;
+  a.partial = partial;
+  const int64_t tiles = (T + kBM - 1) / kBM * splits;
+  if (mma_n <= 64) return launch<__nv_bfloat16, 64, 1, EPI_PARTIAL, 9>(L, ta, tb, tb, a, tiles);
+  if (mma_n <= 128) return launch<__nv_bfloat16, 128, 1, EPI_PARTIAL, 6>(L, ta, tb, tb, a, tiles);
+  return launch<__nv_bfloat16, 256, 1, EPI_PARTIAL, kStages>(L, ta, tb, tb, a, tiles);
+}
+
 constexpr int kMxStages = 5;
 
 cudaError_t expert_gateup_mxfp4(const Launch& L, int64_t R, int D, int F, int E, const void* x_perm,

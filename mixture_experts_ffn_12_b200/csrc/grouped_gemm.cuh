@@ -16,6 +16,8 @@
 //                     done in the down projection's epilogue.
 //   EPI_TOPK          router: logits = C + b[n]; the k largest per row (ties -> lower
 //                     expert index) and the softmax over them.
+//   EPI_PARTIAL       router, K split: the tile's column block index selects one of
+//                     k_splits K ranges; the fp32 partial logits go to `partial`.
 //
 // Kernel organisation (one CTA per SM, 192 threads):
 //   warp 0      TMA producer: A tile [128 x 128 B] and B tile(s) [TN x 128 B] per
@@ -43,7 +45,7 @@
 
 namespace moe {
 
-enum EpiKind : int { EPI_SWIGLU = 0, EPI_BIAS = 1, EPI_BIAS_WSCATTER = 2, EPI_TOPK = 3 };
+enum EpiKind : int { EPI_SWIGLU = 0, EPI_BIAS = 1, EPI_BIAS_WSCATTER = 2, EPI_TOPK = 3, EPI_PARTIAL = 4 };
 
 struct GemmArgs {
   const int32_t* group_off;    // [G+1] row offsets of the groups in A; nullptr = one group of m_total rows
@@ -65,6 +67,8 @@ struct GemmArgs {
   unsigned long long wait_limit_ns;
   const uint8_t* scale0;       // MXFP4: E8M0 scales of B0 / B1, [G, n_out, k_dim / 32]
   const uint8_t* scale1;
+  int k_splits;                // EPI_PARTIAL: K ranges; column block index = K range
+  float* partial;              // EPI_PARTIAL: [k_splits, m_total, n_out] fp32
 };
 
 constexpr int kBM = 128;           // rows per tile (MMA M)
@@ -232,6 +236,22 @@ __device__ __forceinline__ void epi_topk(uint32_t tbase, int row, bool rvalid, c
   }
 }
 
+__device__ __forceinline__ void epi_partial(uint32_t tbase, int row, bool rvalid, const TileInfo& ti,
+                                            const GemmArgs& a, int split) {
+  float* out = a.partial + (static_cast<size_t>(split) * a.m_total + row) * a.n_out;
+#pragma unroll 1
+  for (int c = 0; c < a.mma_n; c += 8) {
+    float v[8];
+    tmem_ld8(tbase + c, v);
+    tmem_ld_wait();
+    if (rvalid) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (c + j < a.n_out) out[c + j] = v[j];
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
@@ -261,9 +281,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = threadIdx.x & 31;
   const bool single = args.group_off == nullptr;
   const int G = single ? 1 : args.num_groups;
-  const int NT = (args.n_out + TN - 1) / TN;
+  const int NT = (EPI == EPI_PARTIAL) ? args.k_splits : (args.n_out + TN - 1) / TN;
   const int KB = (args.k_dim + BK - 1) / BK;
+  const int KBS = (EPI == EPI_PARTIAL) ? (KB + args.k_splits - 1) / args.k_splits : KB;   // k-blocks per range
   const uint64_t lim = args.wait_limit_ns;
+  // k-block range of a tile: all of K, or (EPI_PARTIAL) the range of its column block index
+  auto kb_range = [&](const TileInfo& ti, int& b, int& e) {
+    if (EPI == EPI_PARTIAL) {
+      const int split = ti.n0 / TN;
+      b = split * KBS;
+      e = min(KB, b + KBS);
+    } else {
+      b = 0;
+      e = KB;
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -327,20 +359,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const int mma_n = (EPI == EPI_TOPK) ? args.mma_n : TN * NB;
+      const int mma_n = (EPI == EPI_TOPK || EPI == EPI_PARTIAL) ? args.mma_n : TN * NB;
       const uint32_t tx_bytes = LY::A_BYTES + static_cast<uint32_t>(mma_n) * kRowBytes;
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_par = 0;
       bool ok = true;
       for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
         const TileInfo ti = decode_tile(i, tile_off, goff, G, NT, TN);
-        for (int kb = 0; kb < KB; ++kb) {
+        int kb0, kb1;
+        kb_range(ti, kb0, kb1);
+        const int b_row = (EPI == EPI_PARTIAL) ? 0 : ti.n0;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], tx_bytes);
           uint8_t* sa = smem + s * LY::STAGE_BYTES;
           uint8_t* sb = sa + LY::A_BYTES;
           tma_load_2d(sa, &tmA, &full[s], kb * BK, ti.m0);
-          tma_load_3d(sb, &tmB0, &full[s], kb * BK, ti.n0, ti.g);
+          tma_load_3d(sb, &tmB0, &full[s], kb * BK, b_row, ti.g);
           if (NB == 2) tma_load_3d(sb + TN * kRowBytes, &tmB1, &full[s], kb * BK, ti.n0, ti.g);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
@@ -360,7 +395,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const int mma_n = (EPI == EPI_TOPK) ? args.mma_n : TN * NB;
+      const int mma_n = (EPI == EPI_TOPK || EPI == EPI_PARTIAL) ? args.mma_n : TN * NB;
       const uint32_t idesc = make_idesc(kBM, mma_n, kTF32 ? 2u : 1u);
       int s = 0, it = 0;
       uint32_t ph = 0;
@@ -368,10 +403,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int i = blockIdx.x; ok && i < total; i += gridDim.x, ++it) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
+        int kb0, kb1;
+        kb_range(decode_tile(i, tile_off, goff, G, NT, TN), kb0, kb1);
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, lim)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag, lim)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * LY::STAGE_BYTES);
@@ -379,7 +416,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < KSTEPS; ++kk)
             tc_mma<kTF32>(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
-                          (kb | kk) != 0 ? 1u : 0u);
+                          (kb != kb0 || kk != 0) ? 1u : 0u);
           tc_commit(&empty[s]);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
         }
@@ -415,6 +452,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if constexpr (EPI == EPI_SWIGLU) epi_swiglu<T, TN>(tbase, row, rvalid, ti, args);
       else if constexpr (EPI == EPI_BIAS) epi_bias<T, TN, false>(tbase, row, rvalid, ti, args);
       else if constexpr (EPI == EPI_BIAS_WSCATTER) epi_bias<T, TN, true>(tbase, row, rvalid, ti, args);
+      else if constexpr (EPI == EPI_PARTIAL) epi_partial(tbase, row, rvalid, ti, args, ti.n0 / TN);
       else epi_topk<T>(tbase, row, rvalid, args);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);

@@ -20,9 +20,12 @@ struct Launch {
   unsigned long long wait_limit_ns;
 };
 
-// Router + top-k + softmax.  ids/w are [T, k].
+// Router + top-k + softmax.  ids/w are [T, k].  `partial` (router_partial_bytes of
+// scratch, may be null) lets large bf16 batches split K across more CTAs.
 cudaError_t router_topk(const Launch& L, bool bf16, int64_t T, int D, int E, int k, const void* x,
-                        const void* w_router, const void* b_router, int32_t* ids, float* w);
+                        const void* w_router, const void* b_router, int32_t* ids, float* w,
+                        float* partial = nullptr);
+size_t router_partial_bytes(int64_t T, int E);
 
 // Scratch (int32 words) the permute needs for T tokens and E experts.
 size_t permute_scratch_words(int64_t T, int E);

@@ -61,7 +61,7 @@ size_t elem_size(const moe_config_t* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
 size_t ffn_ws_bytes(const moe_config_t*, int64_t) { return 0; }
 
 struct Layout {
-  size_t ids, w, off, ros, sor, pscr, xperm, h, ys, ffn, total;
+  size_t ids, w, off, ros, sor, pscr, xperm, h, rpart, ys, ffn, total;
 };
 
 Layout layout(const moe_config_t* c, int64_t T) {
@@ -82,7 +82,11 @@ Layout layout(const moe_config_t* c, int64_t T) {
   // x_perm is dead once gate/up has run: the weighted fp32 expert outputs reuse its region
   L.xperm = take(R * c->hidden_size * (es > 4 ? es : 4));
   L.ys = L.xperm;
-  L.h = take(R * c->intermediate_size * es);
+  // the router's K-split partial logits are dead before gate/up writes h: they share it
+  const size_t h_bytes = R * c->intermediate_size * es;
+  const size_t rpart_bytes = moe::router_partial_bytes(T, c->num_local_experts);
+  L.h = take(h_bytes > rpart_bytes ? h_bytes : rpart_bytes);
+  L.rpart = L.h;
   L.ffn = take(ffn_ws_bytes(c, T));
   L.total = o;
   return L;
@@ -340,7 +344,9 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x
   const int D = cfg->hidden_size, E = cfg->num_local_experts, k = cfg->num_experts_per_tok;
 
   stage_mark(ST_ROUTER, true, L.stream);
-  if (moe::router_topk(L, bf16, T, D, E, k, x, w_router, b_router, ids, w) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::router_topk(L, bf16, T, D, E, k, x, w_router, b_router, ids, w,
+                       reinterpret_cast<float*>(base + LY.rpart)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   stage_mark(ST_ROUTER, false, L.stream);
   stage_mark(ST_DISPATCH, true, L.stream);
   if (moe::permute(L, bf16, T, D, E, k, ids, x, eoff, ros, sor, xperm, pscr) != cudaSuccess) return MOE_ERR_CUDA;

@@ -29,6 +29,7 @@ namespace moe {
 // router, SIMT: one block (16 warps) per token
 // ---------------------------------------------------------------------------
 constexpr int kRouterWarps = 32;   // one block per token: a warp per expert for E <= 32
+constexpr int kRouterSplits = 4;   // K ranges of the tensor-core router inside the fused layer
 
 template <typename T>
 __device__ __forceinline__ float dot_row16(const T* a, const T* b, int D, int lane) {
@@ -63,27 +64,10 @@ __device__ __forceinline__ float dot_row16(const T* a, const T* b, int D, int la
   return acc;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kRouterWarps * 32)
-    router_simt_kernel(const T* __restrict__ x, const T* __restrict__ wr, const T* __restrict__ br, int D, int E,
-                       int k, int32_t* __restrict__ ids, float* __restrict__ wout) {
-  __shared__ float logits[256];
-  const int t = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const T* xr = x + static_cast<size_t>(t) * D;
-  for (int e = warp; e < E; e += kRouterWarps) {
-    const float l = dot_row16<T>(xr, wr + static_cast<size_t>(e) * D, D, lane);
-    if (lane == 0) logits[e] = l + to_f32<T>(br[e]);
-  }
-  __syncthreads();
-  if (warp != 0) return;
-  // each lane holds experts lane, lane+32, ... (E <= 256 -> 8 values)
-  float v[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = e < E ? logits[e] : -INFINITY;
-  }
+// Top-k of the logits one warp holds (lane i holds experts i, i+32, ...; -inf past E)
+// and the softmax over the selected ones; lane 0 writes ids[0..k) in descending logit
+// order (ties -> lower expert index) and their weights w[0..k).  Clobbers v.
+__device__ __forceinline__ void warp_topk_softmax(float (&v)[8], int lane, int E, int k, int32_t* ids, float* w) {
   float sel_v[8];
   int sel_e[8];
 #pragma unroll
@@ -121,18 +105,82 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
     }
     const float inv = 1.0f / z;
     for (int j = 0; j < k; ++j) {
-      ids[static_cast<size_t>(t) * k + j] = sel_e[j];
-      wout[static_cast<size_t>(t) * k + j] = ex[j] * inv;
+      ids[j] = sel_e[j];
+      w[j] = ex[j] * inv;
     }
   }
 }
 
+// Fused-layer router tail: sum of the K-range partial logits + router bias, then
+// top-k and softmax.  One warp per token.
+template <typename T>
+__global__ void __launch_bounds__(256) router_topk_partials_kernel(const float* __restrict__ partial, int splits,
+                                                                   const T* __restrict__ br, int Tn, int E, int k,
+                                                                   int32_t* __restrict__ ids,
+                                                                   float* __restrict__ wout) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= Tn) return;
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    float acc = -INFINITY;
+    if (e < E) {
+      acc = 0.0f;
+      for (int sp = 0; sp < splits; ++sp) acc += partial[(static_cast<size_t>(sp) * Tn + t) * E + e];
+      acc += to_f32<T>(br[e]);
+    }
+    v[i] = acc;
+  }
+  warp_topk_softmax(v, lane, E, k, ids + static_cast<size_t>(t) * k, wout + static_cast<size_t>(t) * k);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRouterWarps * 32)
+    router_simt_kernel(const T* __restrict__ x, const T* __restrict__ wr, const T* __restrict__ br, int D, int E,
+                       int k, int32_t* __restrict__ ids, float* __restrict__ wout) {
+  __shared__ float logits[256];
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const T* xr = x + static_cast<size_t>(t) * D;
+  for (int e = warp; e < E; e += kRouterWarps) {
+    const float l = dot_row16<T>(xr, wr + static_cast<size_t>(e) * D, D, lane);
+    if (lane == 0) logits[e] = l + to_f32<T>(br[e]);
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  // each lane holds experts lane, lane+32, ... (E <= 256 -> 8 values)
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? logits[e] : -INFINITY;
+  }
+  warp_topk_softmax(v, lane, E, k, ids + static_cast<size_t>(t) * k, wout + static_cast<size_t>(t) * k);
+}
+
 cudaError_t router_tc(const Launch& L, int64_t T, int D, int E, int k, const void* x, const void* w_router,
-                      const void* b_router, int32_t* ids, float* w);   // gemm_launch.cu
+                      const void* b_router, int32_t* ids, float* w);   // gemm_launch.cuh
+cudaError_t router_tc_partial(const Launch& L, int64_t T, int D, int E, int splits, const void* x,
+                              const void* w_router, float* partial);    // gemm_launch.cuh
+
+size_t router_partial_bytes(int64_t T, int E) { return static_cast<size_t>(kRouterSplits) * T * E * 4; }
 
 cudaError_t router_topk(const Launch& L, bool bf16, int64_t T, int D, int E, int k, const void* x,
-                        const void* w_router, const void* b_router, int32_t* ids, float* w) {
+                        const void* w_router, const void* b_router, int32_t* ids, float* w, float* partial) {
   if (T == 0) return cudaSuccess;
+  // every K range must hold at least one 64-element k-block
+  const int kblocks = (D + 63) / 64, per_split = (kblocks + kRouterSplits - 1) / kRouterSplits;
+  if (bf16 && T >= 256 && partial != nullptr && (kRouterSplits - 1) * per_split < kblocks) {
+    // K split over kRouterSplits ranges so that more CTAs stream x, then sum + top-k
+    cudaError_t e = router_tc_partial(L, T, D, E, kRouterSplits, x, w_router, partial);
+    if (e != cudaSuccess) return e;
+    router_topk_partials_kernel<__nv_bfloat16><<<static_cast<unsigned>((T + 7) / 8), 256, 0, L.stream>>>(
+        partial, kRouterSplits, static_cast<const __nv_bfloat16*>(b_router), static_cast<int>(T), E, k, ids, w);
+    count_launch();
+    return cudaGetLastError();
+  }
   if (bf16 && T >= 256) return router_tc(L, T, D, E, k, x, w_router, b_router, ids, w);
   const dim3 grid(static_cast<unsigned>(T));
   if (bf16)
