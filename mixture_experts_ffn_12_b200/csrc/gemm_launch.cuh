@@ -15,6 +15,7 @@
 #include "decode_gemm.cuh"
 #include "grouped_gemm_pair.cuh"
 #include "grouped_gemm_pair_mx.cuh"
+#include "grouped_gemm_wm_pair.cuh"
 #include "internal.h"
 #include "simt_gemm.cuh"
 
@@ -145,17 +146,44 @@ static cudaError_t launch_pair_mx(const Launch& L, const CUtensorMap& a, const C
   return cudaGetLastError();
 }
 
+// CTA pairs with the weights in M (cluster of 2; grid = 2 x clusters).
+template <int EPI>
+static cudaError_t launch_wm_pair(const Launch& L, const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x,
+                                  const CUtensorMap& x16, const GemmArgs& args, int64_t max_units) {
+  if (max_units <= 0) return cudaSuccess;
+  auto kern = grouped_gemm_wm_pair_kernel<EPI, kWmStages>;
+  constexpr int smem = WmLayout::smem_bytes(kWmStages);
+  static_assert(smem <= 232448, "shared memory budget");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static std::mutex mu;
+  static uint64_t configured = 0;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (dev >= 64 || !((configured >> dev) & 1u)) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) configured |= uint64_t(1) << dev;
+    }
+  }
+  const int clusters = static_cast<int>(std::min<int64_t>(max_units, L.num_sms / 2));
+  kern<<<2 * clusters, kGemmThreads, smem, L.stream>>>(w0, w1, x, x16, args);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // Expert-GEMM variant (moe_set_expert_gemm_variant): 0 = by size, 1 = single-CTA
-// tiles, 2 = CTA-pair tiles, 3 = weight-stationary decode kernel.
+// tiles, 2 = CTA-pair tiles, 3 = weight-stationary decode kernel, 4 = CTA pairs
+// with the weights in M.
 inline std::atomic<int> g_gemm_variant{0};
 
-enum GemmKind { GK_SINGLE = 1, GK_PAIR = 2, GK_DECODE = 3 };
+enum GemmKind { GK_SINGLE = 1, GK_PAIR = 2, GK_DECODE = 3, GK_WM_PAIR = 4 };
 
 // By default: the decode kernel while experts average at most 16 rows (the
 // layer is a weight stream), single-CTA 128-row tiles otherwise.
 static GemmKind gemm_kind(int64_t R, int E) {
   const int v = g_gemm_variant.load();
-  if (v >= 1 && v <= 3) return static_cast<GemmKind>(v);
+  if (v >= 1 && v <= 4) return static_cast<GemmKind>(v);
   return R <= int64_t(16) * E ? GK_DECODE : GK_SINGLE;
 }
 static bool use_pair(int64_t R, int E) { return gemm_kind(R, E) == GK_PAIR; }
@@ -353,6 +381,14 @@ cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, i
     const int64_t units = (std::min<int64_t>(E, R) + R / kDecTok) * ((F + 63) / 64);
     return launch_decode<EPI_SWIGLU>(L, wg, wu, tx, a, units);
   }
+  if (gemm_kind(R, E) == GK_WM_PAIR) {
+    CUtensorMap wg, wu, tx16;
+    if ((e = make_tmap(&wg, w.w_gate, false, D, F, E, 16)) != cudaSuccess) return e;
+    if ((e = make_tmap(&wu, w.w_up, false, D, F, E, 16)) != cudaSuccess) return e;
+    if ((e = make_tmap(&tx16, x_perm, false, D, R, 0, 16)) != cudaSuccess) return e;
+    const int64_t units = ((R + kWmTok - 1) / kWmTok + E) * ((F + 127) / 128);
+    return launch_wm_pair<EPI_SWIGLU>(L, wg, wu, ta, tx16, a, units);
+  }
   if (use_pair(R, E)) {
     const int64_t ptiles = ((R + kPairBM - 1) / kPairBM + E) * ((F + kTNHalf - 1) / kTNHalf);
     return launch_pair<kTNHalf, EPI_SWIGLU, kPairStages>(L, ta, tg, tu, a, ptiles);
@@ -408,6 +444,14 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
     const int64_t units = (std::min<int64_t>(E, R) + R / kDecTok) * ((D + 127) / 128);
     if (slot_of_row != nullptr) return launch_decode<EPI_BIAS_WSCATTER>(L, wd, wd, th, a, units);
     return launch_decode<EPI_BIAS>(L, wd, wd, th, a, units);
+  }
+  if (gemm_kind(R, E) == GK_WM_PAIR) {
+    CUtensorMap wd, th16;
+    if ((e = make_tmap(&wd, w.w_down, false, F, D, E, 128)) != cudaSuccess) return e;
+    if ((e = make_tmap(&th16, h, false, F, R, 0, 16)) != cudaSuccess) return e;
+    const int64_t units = ((R + kWmTok - 1) / kWmTok + E) * ((D + 255) / 256);
+    if (slot_of_row != nullptr) return launch_wm_pair<EPI_BIAS_WSCATTER>(L, wd, wd, ta, th16, a, units);
+    return launch_wm_pair<EPI_BIAS>(L, wd, wd, ta, th16, a, units);
   }
   const bool pair = use_pair(R, E);
   if ((e = make_tmap(&tb, w.w_down, !bf16, F, D, E, pair ? kTNHalf : kTNDown)) != cudaSuccess) return e;

@@ -113,22 +113,32 @@ __device__ __forceinline__ void warp_topk_softmax(float (&v)[8], int lane, int E
 
 // Fused-layer router tail: sum of the K-range partial logits + router bias, then
 // top-k and softmax.  One warp per token.
-template <typename T>
-__global__ void __launch_bounds__(256) router_topk_partials_kernel(const float* __restrict__ partial, int splits,
+template <typename T, int SPLITS>
+__global__ void __launch_bounds__(256) router_topk_partials_kernel(const float* __restrict__ partial,
                                                                    const T* __restrict__ br, int Tn, int E, int k,
                                                                    int32_t* __restrict__ ids,
                                                                    float* __restrict__ wout) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= Tn) return;
+  // all loads first (they are independent), then the sums in split order
+  float p[8][SPLITS];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+#pragma unroll
+    for (int sp = 0; sp < SPLITS; ++sp)
+      p[i][sp] = e < E ? __ldcg(partial + (static_cast<size_t>(sp) * Tn + t) * E + e) : 0.0f;
+  }
   float v[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = lane + 32 * i;
     float acc = -INFINITY;
     if (e < E) {
-      acc = 0.0f;
-      for (int sp = 0; sp < splits; ++sp) acc += partial[(static_cast<size_t>(sp) * Tn + t) * E + e];
+      acc = p[i][0];
+#pragma unroll
+      for (int sp = 1; sp < SPLITS; ++sp) acc += p[i][sp];
       acc += to_f32<T>(br[e]);
     }
     v[i] = acc;
@@ -176,8 +186,8 @@ cudaError_t router_topk(const Launch& L, bool bf16, int64_t T, int D, int E, int
     // K split over kRouterSplits ranges so that more CTAs stream x, then sum + top-k
     cudaError_t e = router_tc_partial(L, T, D, E, kRouterSplits, x, w_router, partial);
     if (e != cudaSuccess) return e;
-    router_topk_partials_kernel<__nv_bfloat16><<<static_cast<unsigned>((T + 7) / 8), 256, 0, L.stream>>>(
-        partial, kRouterSplits, static_cast<const __nv_bfloat16*>(b_router), static_cast<int>(T), E, k, ids, w);
+    router_topk_partials_kernel<__nv_bfloat16, kRouterSplits><<<static_cast<unsigned>((T + 7) / 8), 256, 0, L.stream>>>(
+        partial, static_cast<const __nv_bfloat16*>(b_router), static_cast<int>(T), E, k, ids, w);
     count_launch();
     return cudaGetLastError();
   }

@@ -138,15 +138,42 @@ def test_expert_ffn(api, spec):
     check_stored(f64(yp), ry, tol, spec.dtype == "bf16")
 
 
+@pytest.mark.parametrize("variant", [1, 2, 4], ids=["single_cta", "cta_pair", "wm_pair"])
+@pytest.mark.parametrize("spec", [RAGGED_BF16, WIDE_K, PAIR_RAGGED], ids=lambda s: s.name)
+def test_expert_ffn_each_gemm_variant(api, spec, variant):
+    """moe_expert_ffn (bf16 down rows, no weighting) through each prefill GEMM kernel."""
+    layer = layer_for(spec)
+    ids, w, off, ros, sor, xp = _expert_inputs(spec, layer, api)
+    d = dev({k: v for k, v in layer.items() if k not in ("x",)}, api)
+    cfg = api.config_from_spec(spec)
+    api.set_expert_gemm_variant(variant)
+    try:
+        h, yp = api.expert_ffn(cfg, api.to_torch(xp).cuda(), torch.from_numpy(off).cuda(),
+                               api.expert_weights_from(d))
+        torch.cuda.synchronize()
+    finally:
+        api.set_expert_gemm_variant(0)
+    assert api.last_device_error() == 0
+    rh, ry = O.expert_ffn(xp, off, layer, spec.limit, spec.alpha)
+    check_stored(f64(h), rh, tol_for(spec), True)
+    check_stored(f64(yp), ry, tol_for(spec), True)
+
+
+@pytest.mark.parametrize("variant", [0, 4], ids=["default", "wm_pair"])
 @pytest.mark.parametrize("spec", [W.GPTOSS20B_PREFILL], ids=lambda s: s.name)
-def test_expert_ffn_full_size_some_experts(api, spec):
+def test_expert_ffn_full_size_some_experts(api, spec, variant):
     """GPT-OSS-20B-shaped gate/up/down on all 16384 routed rows; the oracle checks three whole experts."""
     layer = layer_for(spec)
     ids, w, off, ros, sor, xp = _expert_inputs(spec, layer, api)
     d = dev({k: v for k, v in layer.items() if k not in ("x",)}, api)
     cfg = api.config_from_spec(spec)
-    h, yp = api.expert_ffn(cfg, api.to_torch(xp).cuda(), torch.from_numpy(off).cuda(), api.expert_weights_from(d))
-    torch.cuda.synchronize()
+    api.set_expert_gemm_variant(variant)
+    try:
+        h, yp = api.expert_ffn(cfg, api.to_torch(xp).cuda(), torch.from_numpy(off).cuda(),
+                               api.expert_weights_from(d))
+        torch.cuda.synchronize()
+    finally:
+        api.set_expert_gemm_variant(0)
     assert api.last_device_error() == 0
     for e in (0, 13, spec.E - 1):
         a, b = int(off[e]), int(off[e + 1])
@@ -203,6 +230,20 @@ def test_layer_forward_all_tokens(api, spec):
 @pytest.mark.parametrize("spec", [W.GPTOSS20B_PREFILL, W.GPTOSS20B_MXFP4, W.GPTOSS120B_SKEWED],
                          ids=lambda s: s.name)
 def test_layer_forward_full_size_sampled(api, spec):
+    _full_size_sampled(api, spec)
+
+
+@pytest.mark.parametrize("spec", [W.GPTOSS20B_PREFILL, W.GPTOSS120B_SKEWED], ids=lambda s: s.name)
+def test_layer_forward_full_size_sampled_wm_pair(api, spec):
+    """The full-size bf16 layers through the CTA-pair kernels with the weights in M."""
+    api.set_expert_gemm_variant(4)
+    try:
+        _full_size_sampled(api, spec)
+    finally:
+        api.set_expert_gemm_variant(0)
+
+
+def _full_size_sampled(api, spec):
     layer = layer_for(spec)
     y, gid, _ = _run_layer(api, spec, layer)
     # routing: every token, bit-exact
@@ -233,12 +274,13 @@ def test_layer_forward_repeatable(api):
     assert torch.equal(y1, y2)
 
 
-@pytest.mark.parametrize("variant", [1, 2, 3], ids=["single_cta", "cta_pair", "decode"])
+@pytest.mark.parametrize("variant", [1, 2, 3, 4], ids=["single_cta", "cta_pair", "decode", "wm_pair"])
 @pytest.mark.parametrize("spec", [RAGGED_BF16, PAIR_RAGGED, W.gptoss20b_decode(8)], ids=lambda s: s.name)
 def test_layer_forward_each_gemm_variant(api, spec, variant):
     """Every bf16 expert-GEMM kernel on the same layer: single-CTA 128-row tiles, CTA pairs
-    (256 rows), and the weight-stationary decode kernel (token chunks of 32, so experts with
-    more rows run several chunks)."""
+    (256 rows), the weight-stationary decode kernel (token chunks of 32, so experts with
+    more rows run several chunks), and CTA pairs with the weights in M (token tiles of up
+    to 256 columns, ragged last tiles rounded to 16)."""
     layer = layer_for(spec)
     api.set_expert_gemm_variant(variant)
     try:
