@@ -117,9 +117,11 @@ MOE_API moe_status_t moe_config_check(const moe_config_t* cfg);
  * scratch).  0 when T == 0; (size_t)-1 if cfg is invalid. */
 MOE_API size_t moe_permute_workspace_size(const moe_config_t* cfg, int64_t T);
 
-/* Bytes of workspace moe_expert_ffn needs: 0 for every supported configuration
- * (MXFP4 weights are dequantised inside the GEMM mainloop); kept so callers can
- * size a workspace without knowing that.  (size_t)-1 if cfg is invalid. */
+/* Bytes of workspace moe_expert_ffn needs: 0 for dense weights; for MXFP4 the
+ * E8M0 scales of the three projections relaid for TMA (per matrix with N rows
+ * and reduction length K: E * ceil(K/64) * N * 2 bytes, each region rounded up
+ * to 256 bytes), rewritten from the caller's scales on every call.  Independent
+ * of T.  (size_t)-1 if cfg is invalid. */
 MOE_API size_t moe_expert_ffn_workspace_size(const moe_config_t* cfg, int64_t T);
 
 /* Bytes of workspace moe_layer_forward needs for T tokens: routing ids and
@@ -181,7 +183,8 @@ MOE_API moe_status_t moe_permute_noalloc(const moe_config_t* cfg, int64_t T, con
  * Computed on the tcgen05 tensor cores with fp32 accumulation from bf16
  * operands (MXFP4 weights are decoded to bf16 in shared memory inside the GEMM
  * mainloop; fp32 layers run in fp32 FMA).  ws: moe_expert_ffn_workspace_size
- * bytes (may be NULL when that is 0). */
+ * bytes, 16-byte aligned (may be NULL when that is 0); MOE_ERR_WORKSPACE if it
+ * is missing or too small. */
 MOE_API moe_status_t moe_expert_ffn(const moe_config_t* cfg, int64_t T, const void* x_perm, const int32_t* expert_off,
                             const moe_expert_weights_t* weights, void* h, void* y_perm, void* ws, size_t ws_bytes,
                             void* stream);

@@ -244,8 +244,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t cta_addr, uint32_t rank
   return r;
 }
 
+// Arrive on an mbarrier of a CTA of this cluster (default .release.cta semantics).
+// Writes the arrival must publish to the tensor core are fenced by the caller
+// (fence.proxy.async); a .release.cluster arrive here costs about a microsecond
+// per call, which in a per-K-step handshake starves the MMA.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {

@@ -70,6 +70,21 @@ static cudaError_t make_tmap_packed(CUtensorMap* m, const void* ptr, uint64_t K,
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Relaid MXFP4 scales: [groups][KB][2 * rows] bytes, boxes of box_bytes x 1 x 1, no swizzle.
+static cudaError_t make_tmap_scales(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t KB, uint64_t groups,
+                                   uint32_t box_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {2 * rows, KB, groups};
+  const cuuint64_t strides[2] = {2 * rows, 2 * rows * KB};
+  const cuuint32_t box[3] = {box_bytes, 1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <typename T, int TN, int NB, int EPI, int STAGES>
 static cudaError_t launch(const Launch& L, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                           const GemmArgs& args, int64_t max_tiles) {
@@ -123,7 +138,8 @@ static cudaError_t launch_pair(const Launch& L, const CUtensorMap& a, const CUte
 
 template <int TNH, int EPI, int STAGES>
 static cudaError_t launch_pair_mx(const Launch& L, const CUtensorMap& a, const CUtensorMap& p0, const CUtensorMap& p1,
-                                  const GemmArgs& args, int64_t max_tiles) {
+                                  const CUtensorMap& s0, const CUtensorMap& s1, const GemmArgs& args,
+                                  int64_t max_tiles) {
   if (max_tiles <= 0) return cudaSuccess;
   auto kern = grouped_gemm_pair_mx_kernel<TNH, EPI, STAGES>;
   constexpr int smem = PairMxLayout<TNH>::smem_bytes(STAGES);
@@ -141,7 +157,7 @@ static cudaError_t launch_pair_mx(const Launch& L, const CUtensorMap& a, const C
     }
   }
   const int clusters = static_cast<int>(std::min<int64_t>(max_tiles, L.num_sms / 2));
-  kern<<<2 * clusters, kMxThreads, smem, L.stream>>>(a, p0, p1, args);
+  kern<<<2 * clusters, kMxThreads, smem, L.stream>>>(a, p0, p1, s0, s1, args);
   count_launch();
   return cudaGetLastError();
 }
@@ -281,14 +297,36 @@ cudaError_t router_tc_partial(const Launch& L, int64_t T, int D, int E, int spli
 
 constexpr int kMxStages = 5;
 
+size_t mx_scale_bytes(int rows, int K, int E) {
+  return static_cast<size_t>(E) * ((K + 63) / 64) * rows * 2;
+}
+
+cudaError_t mx_scale_relayout(const Launch& L, int D, int F, int E, const ExpertWeights& w, uint8_t* s_gate,
+                              uint8_t* s_up, uint8_t* s_down) {
+  MxScaleJob job{};
+  job.src[0] = w.s_gate; job.dst[0] = s_gate; job.rows[0] = F; job.kdim[0] = D;
+  job.src[1] = w.s_up;   job.dst[1] = s_up;   job.rows[1] = F; job.kdim[1] = D;
+  job.src[2] = w.s_down; job.dst[2] = s_down; job.rows[2] = D; job.kdim[2] = F;
+  job.groups = E;
+  const int64_t most = std::max(mx_scale_bytes(F, D, E), mx_scale_bytes(D, F, E)) / 2;
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>((most + 255) / 256, int64_t(8) * L.num_sms)), 3);
+  mx_scale_relayout_kernel<<<grid, 256, 0, L.stream>>>(job);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t expert_gateup_mxfp4(const Launch& L, int64_t R, int D, int F, int E, const void* x_perm,
-                                const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h) {
+                                const int32_t* expert_off, const ExpertWeights& w, const uint8_t* s_gate2,
+                                const uint8_t* s_up2, float limit, float alpha, void* h) {
   if (R == 0) return cudaSuccess;
-  CUtensorMap ta, pg, pu;
+  CUtensorMap ta, pg, pu, sg, su;
   cudaError_t e;
+  const int KB = (D + 63) / 64;
   if ((e = make_tmap(&ta, x_perm, false, D, R, 0, kBM)) != cudaSuccess) return e;
   if ((e = make_tmap_packed(&pg, w.w_gate, D, F, E, kTNHalf)) != cudaSuccess) return e;
   if ((e = make_tmap_packed(&pu, w.w_up, D, F, E, kTNHalf)) != cudaSuccess) return e;
+  if ((e = make_tmap_scales(&sg, s_gate2, F, KB, E, 2 * kTNHalf)) != cudaSuccess) return e;
+  if ((e = make_tmap_scales(&su, s_up2, F, KB, E, 2 * kTNHalf)) != cudaSuccess) return e;
   GemmArgs a = base_args(L);
   a.group_off = expert_off;
   a.num_groups = E;
@@ -301,20 +339,20 @@ cudaError_t expert_gateup_mxfp4(const Launch& L, int64_t R, int D, int F, int E,
   a.alpha = alpha;
   a.out = h;
   a.ldo = F;
-  a.scale0 = w.s_gate;
-  a.scale1 = w.s_up;
   const int64_t ptiles = ((R + kPairBM - 1) / kPairBM + E) * ((F + kTNHalf - 1) / kTNHalf);
-  return launch_pair_mx<kTNHalf, EPI_SWIGLU, kMxStages>(L, ta, pg, pu, a, ptiles);
+  return launch_pair_mx<kTNHalf, EPI_SWIGLU, kMxStages>(L, ta, pg, pu, sg, su, a, ptiles);
 }
 
 cudaError_t expert_down_mxfp4(const Launch& L, int64_t R, int D, int F, int E, const void* h,
-                              const int32_t* expert_off, const ExpertWeights& w, const int32_t* slot_of_row,
-                              const float* topk_w, void* out) {
+                              const int32_t* expert_off, const ExpertWeights& w, const uint8_t* s_down2,
+                              const int32_t* slot_of_row, const float* topk_w, void* out) {
   if (R == 0) return cudaSuccess;
-  CUtensorMap ta, pd;
+  CUtensorMap ta, pd, sd;
   cudaError_t e;
+  const int KB = (F + 63) / 64;
   if ((e = make_tmap(&ta, h, false, F, R, 0, kBM)) != cudaSuccess) return e;
   if ((e = make_tmap_packed(&pd, w.w_down, F, D, E, kTNHalf)) != cudaSuccess) return e;
+  if ((e = make_tmap_scales(&sd, s_down2, D, KB, E, 2 * kTNHalf)) != cudaSuccess) return e;
   GemmArgs a = base_args(L);
   a.group_off = expert_off;
   a.num_groups = E;
@@ -326,12 +364,10 @@ cudaError_t expert_down_mxfp4(const Launch& L, int64_t R, int D, int F, int E, c
   a.ldo = D;
   a.slot_of_row = slot_of_row;
   a.topk_w = topk_w;
-  a.scale0 = w.s_down;
-  a.scale1 = w.s_down;
   const int64_t ptiles = ((R + kPairBM - 1) / kPairBM + E) * ((D + 2 * kTNHalf - 1) / (2 * kTNHalf));
   if (slot_of_row != nullptr)
-    return launch_pair_mx<kTNHalf, EPI_BIAS_WSCATTER, kMxStages>(L, ta, pd, pd, a, ptiles);
-  return launch_pair_mx<kTNHalf, EPI_BIAS, kMxStages>(L, ta, pd, pd, a, ptiles);
+    return launch_pair_mx<kTNHalf, EPI_BIAS_WSCATTER, kMxStages>(L, ta, pd, pd, sd, sd, a, ptiles);
+  return launch_pair_mx<kTNHalf, EPI_BIAS, kMxStages>(L, ta, pd, pd, sd, sd, a, ptiles);
 }
 
 cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,

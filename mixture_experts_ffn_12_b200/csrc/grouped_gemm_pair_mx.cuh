@@ -1,36 +1,53 @@
 // CTA-pair grouped GEMM with MXFP4 expert weights dequantised inside the mainloop.
 //
-// Same tiles, roles and epilogues as grouped_gemm_pair.cuh, plus four converter
-// warps per CTA.  Per stage each CTA receives, by TMA, its 128 rows of A (bf16,
-// 128-byte swizzle) and its 120 rows of packed E2M1 weights (32 bytes = 64 codes
-// per row); the converters turn the packed rows into the bf16 swizzled tile the
-// MMA reads, each value being the E2M1 code times the row's E8M0 block scale
-// 2^(s-127) for its 32-element block along K (OCP MX encoding: code bit 3 sign,
-// bits 2..1 exponent with bias 1, bit 0 mantissa; element 2i in the low nibble of
-// byte i).  Every decoded value is a bf16 number, so the MMA sees exactly the
-// dequantised weights.  The leader's MMA waits for both CTAs' A bytes (`full`) and
-// both CTAs' converted halves (`conv`, 8 warp arrivals).
+// Same tiles, MMA and epilogues as grouped_gemm_pair.cuh; the weight half each
+// CTA feeds the MMA is decoded from MXFP4 in shared memory by converter warps.
+// MX encoding (OCP MX): E2M1 codes (bit 3 sign, bits 2..1 exponent with bias 1,
+// bit 0 mantissa; element 2i in the low nibble of byte i) times the E8M0 scale
+// 2^(s-127) of their 32-element block along K.  Every decoded value is a bf16
+// number, so the MMA sees exactly the dequantised weights.
 //
-// Scale bytes (90 per row for K = 2880) are read from global memory by the
-// converters, one k-block ahead, since rows that are not a multiple of 16 bytes
-// cannot be described to TMA.
+// The packed weights travel on a ring of their own, decoupled from the MMA
+// stages: a packed slot holds one 64-wide K step of this CTA's 120 weight rows
+// (32 bytes each) and their 240 scale bytes, both loaded by TMA, and the ring is
+// 16 slots deep, so packed data is resident long before the MMA needs it.  The
+// converters wait for a packed slot and for the MMA stage's weight tile to be
+// free, decode into it, fence the generic-proxy stores for the tensor core and
+// arrive on the leader's `conv` barrier (one arrival per converter warp of the pair); the
+// leader's MMA waits for `full` (both CTAs' activation rows, TMA) and `conv`.
+// Scales are read from a copy relaid as [E][K/64][N][2] (moe_abi's workspace,
+// written by mx_scale_relayout_kernel each call), because rows of K/32 bytes are
+// not a multiple of 16 bytes and cannot be described to TMA as they are stored.
+//
+// Roles (480 threads per CTA):
+//   warp 0      activation producer (TMA, both CTAs, bytes counted on the leader)
+//   warp 1      TMEM; the leader's lane 0 issues the pair MMAs
+//   warps 2-5   epilogue (this CTA's 128 accumulator rows)
+//   warp 6      packed-weight producer (TMA into the packed ring, this CTA)
+//   warps 7-14  converters (two per SM sub-partition, so one's latency hides the other's)
 #pragma once
 
 #include "grouped_gemm_pair.cuh"
 
 namespace moe {
 
-constexpr int kMxThreads = 320;     // 6 warps as in the bf16 kernels + 4 converter warps
-constexpr int kMxConvThreads = 128;
+constexpr int kMxConvWarp0 = 7;     // first converter warp
+constexpr int kMxConvWarps = 8;
+constexpr int kMxThreads = (kMxConvWarp0 + kMxConvWarps) * 32;
+constexpr int kMxPackSlots = 16;    // depth of the packed-weight ring
 
 template <int TNH>
 struct PairMxLayout {
   static constexpr int A_BYTES = 128 * kRowBytes;            // bf16 activations
   static constexpr int B_BYTES = TNH * kRowBytes;            // dequantised bf16 weights
-  static constexpr int P_BYTES = (TNH * 32 + 1023) / 1024 * 1024;   // packed E2M1 rows (32 B each)
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int P_BYTES = TNH * 32;                   // packed E2M1 rows of one K step
+  static constexpr int S_BYTES = TNH * 2;                    // their two scale bytes per row
+  static constexpr int SLOT_BYTES = (P_BYTES + S_BYTES + 255) / 256 * 256;
   static constexpr int EXTRA = 1024 + 4096;
-  static constexpr int smem_bytes(int stages) { return stages * STAGE_BYTES + EXTRA; }
+  static constexpr int smem_bytes(int stages) { return stages * STAGE_BYTES + kMxPackSlots * SLOT_BYTES + EXTRA; }
+  static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-byte aligned for the 128-byte swizzle");
+  static_assert(P_BYTES % 16 == 0 && S_BYTES % 16 == 0, "TMA destinations are 16-byte aligned");
 };
 
 // 8 E2M1 codes (one 32-bit word, element i in nibble i) times a bf16 scale -> 8 bf16 in a uint4.
@@ -72,23 +89,62 @@ __device__ __forceinline__ __nv_bfloat162 e8m0_to_bf16x2(uint32_t s) {
   return __halves2bfloat162(h, h);
 }
 
+// Scales [E][N][K/32] -> [E][ceil(K/64)][N][2]: the two scale bytes of K step kb for
+// row n sit at ((g * KB + kb) * N + n) * 2; a missing second block (K % 64 == 32)
+// gets 127 (its codes are zero).  gridDim.y selects one of up to three matrices.
+struct MxScaleJob {
+  const uint8_t* src[3];
+  uint8_t* dst[3];
+  int rows[3];     // N of each matrix
+  int kdim[3];     // K of each matrix
+  int groups;
+};
+
+__global__ void __launch_bounds__(256) mx_scale_relayout_kernel(MxScaleJob job) {
+  const int m = blockIdx.y;
+  const int N = job.rows[m], K = job.kdim[m];
+  const int KS = K / 32, KB = (K + 63) / 64;
+  const int64_t total = static_cast<int64_t>(job.groups) * KB * N;
+  const uint8_t* src = job.src[m];
+  uint16_t* dst = reinterpret_cast<uint16_t*>(job.dst[m]);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int n = static_cast<int>(i % N);
+    const int64_t gk = i / N;
+    const int kb = static_cast<int>(gk % KB);
+    const int64_t g = gk / KB;
+    const uint8_t* row = src + (g * N + n) * KS;
+    const uint32_t lo = row[2 * kb];
+    const uint32_t hi = 2 * kb + 1 < KS ? row[2 * kb + 1] : 127u;
+    dst[i] = static_cast<uint16_t>(lo | (hi << 8));
+  }
+}
+
+// tmA: activations [R, K] (128-row boxes).  tmP0 / tmP1: packed weights [E][N][K/2]
+// (TNH-row boxes of 32 bytes); tmS0 / tmS1: relaid scales [E][KB][2N] (boxes of
+// 2*TNH bytes).  For SwiGLU index 0 is the gate (leader) and 1 the up projection
+// (peer); otherwise both are the down weights and the CTAs take two column blocks.
 template <int TNH, int EPI, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
     grouped_gemm_pair_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP0,
-                                const __grid_constant__ CUtensorMap tmP1, const GemmArgs args) {
+                                const __grid_constant__ CUtensorMap tmP1, const __grid_constant__ CUtensorMap tmS0,
+                                const __grid_constant__ CUtensorMap tmS1, const GemmArgs args) {
   using T = __nv_bfloat16;
   using LY = PairMxLayout<TNH>;
-  constexpr int BK = kRowBytes / 2;        // 64 K elements per stage
+  constexpr int BK = kRowBytes / 2;        // 64 K elements per step
   constexpr int KSTEPS = kRowBytes / 32;
   constexpr int TNO = (EPI == EPI_SWIGLU) ? TNH : 2 * TNH;
+  constexpr int PS = kMxPackSlots;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * LY::STAGE_BYTES);
+  uint8_t* pring = smem + STAGES * LY::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(pring + PS * LY::SLOT_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* pk = empty + STAGES;           // packed rows landed (local)
-  uint64_t* conv = pk + STAGES;            // both CTAs' halves converted (leader, 8 arrivals)
-  uint64_t* tfull = conv + STAGES;
+  uint64_t* conv = empty + STAGES;         // both CTAs' weight halves decoded (leader, 2 x kMxConvWarps arrivals)
+  uint64_t* pfull = conv + STAGES;         // packed slot landed (local, TMA)
+  uint64_t* pempty = pfull + PS;           // packed slot read by the local converter warps
+  uint64_t* tfull = pempty + PS;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -105,15 +161,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
   const int G = args.num_groups;
   const int NT = (args.n_out + TNO - 1) / TNO;
   const int KB = (args.k_dim + BK - 1) / BK;
-  const int KS = args.k_dim / 32;          // scale bytes per weight row
   const uint64_t lim = args.wait_limit_ns;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&pk[s], 1);
-      mbar_init(&conv[s], 8);
+      mbar_init(&conv[s], 2 * kMxConvWarps);
+    }
+    for (int p = 0; p < PS; ++p) {
+      mbar_init(&pfull[p], 1);
+      mbar_init(&pempty[p], kMxConvWarps);
     }
     mbar_init(&tfull[0], 1);
     mbar_init(&tfull[1], 1);
@@ -157,6 +215,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmP0);
       tma_prefetch_desc(&tmP1);
+      tma_prefetch_desc(&tmS0);
+      tma_prefetch_desc(&tmS1);
     }
   } else if (warp == 1) {
     tmem_alloc_pair(tmem_slot, kTmemCols);
@@ -168,13 +228,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = tile_off[G] * NT;
-  // this CTA's half of B: gate (leader) / up (peer) rows for SwiGLU, else two column blocks
-  const void* tmp = (EPI == EPI_SWIGLU && rank == 1) ? static_cast<const void*>(&tmP1)
-                                                      : static_cast<const void*>(&tmP0);
-  const uint8_t* scales = (EPI == EPI_SWIGLU && rank == 1) ? args.scale1 : args.scale0;
+  // this CTA's weight half: gate (leader) / up (peer) rows for SwiGLU, else two column blocks
+  const bool second = EPI == EPI_SWIGLU && rank == 1;
+  const void* tmp = second ? static_cast<const void*>(&tmP1) : static_cast<const void*>(&tmP0);
+  const void* tms = second ? static_cast<const void*>(&tmS1) : static_cast<const void*>(&tmS0);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (both CTAs)
+    // ------------------------------------------------------------ activation producer (both CTAs)
     if (lane == 0) {
       const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
       int s = 0;
@@ -183,15 +243,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
       for (int i = cluster; ok && i < total; i += nclusters) {
         const TileInfo ti = decode_pair_tile(i, tile_off, goff, G, NT, TNO);
         const int a_row = ti.m0 + static_cast<int>(rank) * 128;
-        const int b_row = (EPI == EPI_SWIGLU) ? ti.n0 : ti.n0 + static_cast<int>(rank) * TNH;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) { ok = false; break; }
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * LY::A_BYTES);
-          uint8_t* sa = smem + s * LY::STAGE_BYTES;
-          uint8_t* sp = sa + LY::A_BYTES + LY::B_BYTES;
-          tma_load_2d_pair(sa, &tmA, full_leader + static_cast<uint32_t>(s) * 8u, kb * BK, a_row);
-          mbar_arrive_expect_tx(&pk[s], TNH * 32);
-          tma_load_3d(sp, tmp, &pk[s], kb * 32, b_row, ti.g);
+          tma_load_2d_pair(smem + s * LY::STAGE_BYTES, &tmA, full_leader + static_cast<uint32_t>(s) * 8u, kb * BK,
+                           a_row);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -200,15 +256,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
       if (!ok) {
         *abort_flag = 1;
         flag_error(DEVERR_TIMEOUT);
+        // the peer's barrier cannot be polled from here: give loads in flight time to land
         for (int q = 0; q < 2000; ++q) __nanosleep(1000);
       }
-      // packed loads signal this CTA's own barriers: wait for every one issued
-      for (int q = 0; q < STAGES; ++q)
-        if ((issued >> q) & 1u) {
-          if (!mbar_wait(&pk[q], (issued_par >> q) & 1u, never_flag, kDrainLimitNs)) flag_error(DEVERR_TIMEOUT);
-          if (rank == 0 && !mbar_wait(&full[q], (issued_par >> q) & 1u, never_flag, kDrainLimitNs))
-            flag_error(DEVERR_TIMEOUT);
+      if (rank == 0) {
+        for (int q = 0; q < STAGES; ++q)
+          if ((issued >> q) & 1u)
+            if (!mbar_wait(&full[q], (issued_par >> q) & 1u, never_flag, kDrainLimitNs)) flag_error(DEVERR_TIMEOUT);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ packed-weight producer (both CTAs)
+    if (lane == 0) {
+      int p = 0;
+      uint32_t pph = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      for (int i = cluster; ok && i < total; i += nclusters) {
+        const TileInfo ti = decode_pair_tile(i, tile_off, goff, G, NT, TNO);
+        const int b_row = (EPI == EPI_SWIGLU) ? ti.n0 : ti.n0 + static_cast<int>(rank) * TNH;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&pempty[p], pph ^ 1u, abort_flag, lim)) { ok = false; break; }
+          mbar_arrive_expect_tx(&pfull[p], LY::P_BYTES + LY::S_BYTES);
+          uint8_t* slot = pring + p * LY::SLOT_BYTES;
+          tma_load_3d(slot, tmp, &pfull[p], kb * 32, b_row, ti.g);
+          tma_load_3d(slot + LY::P_BYTES, tms, &pfull[p], 2 * b_row, kb, ti.g);
+          issued |= 1u << p;
+          issued_par = (issued_par & ~(1u << p)) | (pph << p);
+          if (++p == PS) { p = 0; pph ^= 1u; }
         }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag_error(DEVERR_TIMEOUT);
+      }
+      // these loads signal this CTA's own barriers: wait for every one issued
+      for (int q = 0; q < PS; ++q)
+        if ((issued >> q) & 1u)
+          if (!mbar_wait(&pfull[q], (issued_par >> q) & 1u, never_flag, kDrainLimitNs)) flag_error(DEVERR_TIMEOUT);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -227,7 +312,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag, lim)) { ok = false; break; }
-          if (!mbar_wait(&conv[s], ph, abort_flag, lim)) { ok = false; break; }
+          if (!mbar_wait_cluster(&conv[s], ph, abort_flag, lim)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * LY::STAGE_BYTES);
           const uint32_t b_addr = a_addr + LY::A_BYTES;
@@ -283,53 +368,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ converters (both CTAs)
-    const int ct = threadIdx.x - 6 * 32;                 // 0..127
+    constexpr int kRowStep = kMxConvWarps * 4;           // rows r0, r0 + kRowStep, ...
+    const int ct = threadIdx.x - kMxConvWarp0 * 32;      // 0 .. 32 * kMxConvWarps - 1
     const uint32_t conv_leader = mapa_shared(smem_u32(conv), 0);
-    const int c = ct & 7;                                // 16-byte chunk within a row (8 codes)
-    const int r0 = ct >> 3;                              // rows r0, r0 + 16, ...
-    int s = 0;
-    uint32_t ph = 0;
+    const int c = ct & 7;                                // 4-byte chunk of a 32-byte packed row (8 codes)
+    const int r0 = ct >> 3;
+    int s = 0, p = 0;
+    uint32_t ph = 0, pph = 0;
     bool ok = true;
     for (int i = cluster; ok && i < total; i += nclusters) {
-      const TileInfo ti = decode_pair_tile(i, tile_off, goff, G, NT, TNO);
-      const int b_row = (EPI == EPI_SWIGLU) ? ti.n0 : ti.n0 + static_cast<int>(rank) * TNH;
-      // this thread's scale bytes for one k-block: rows r0 + 16 j, block kb * 2 + c / 4
-      const uint8_t* srow = scales + (static_cast<size_t>(ti.g) * args.n_out + b_row) * KS + (c >> 2);
-      uint8_t sc_next[(TNH + 15) / 16];
-#pragma unroll
-      for (int j = 0; j < (TNH + 15) / 16; ++j) {
-        const int r = r0 + 16 * j;
-        sc_next[j] = (r < TNH && b_row + r < args.n_out) ? srow[static_cast<size_t>(r) * KS] : uint8_t(127);
-      }
       for (int kb = 0; kb < KB; ++kb) {
-        uint8_t sc[(TNH + 15) / 16];
-#pragma unroll
-        for (int j = 0; j < (TNH + 15) / 16; ++j) sc[j] = sc_next[j];
-        if (!__all_sync(0xffffffffu, mbar_wait(&pk[s], ph, abort_flag, lim))) { ok = false; break; }
-        const uint8_t* sp = smem + s * LY::STAGE_BYTES + LY::A_BYTES + LY::B_BYTES;
+        // packed slot landed, and the MMA is done with this stage's weight tile
+        if (!__all_sync(0xffffffffu, mbar_wait(&pfull[p], pph, abort_flag, lim))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim))) { ok = false; break; }
+        const uint8_t* sp = pring + p * LY::SLOT_BYTES;
+        const uint8_t* ss = sp + LY::P_BYTES;
         uint8_t* sb = smem + s * LY::STAGE_BYTES + LY::A_BYTES;
 #pragma unroll
-        for (int j = 0; j < (TNH + 15) / 16; ++j) {
-          const int r = r0 + 16 * j;
+        for (int j = 0; j < (TNH + kRowStep - 1) / kRowStep; ++j) {
+          const int r = r0 + kRowStep * j;
           if (r < TNH) {
             const uint32_t w = *reinterpret_cast<const uint32_t*>(sp + r * 32 + c * 4);
-            const uint4 v = mxfp4_decode8(w, e8m0_to_bf16x2(sc[j]));
+            const uint4 v = mxfp4_decode8(w, e8m0_to_bf16x2(ss[r * 2 + (c >> 2)]));
             *reinterpret_cast<uint4*>(sb + r * kRowBytes + ((c ^ (r & 7)) << 4)) = v;
           }
         }
         fence_proxy_async_smem();     // generic-proxy stores -> visible to the tensor core
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(conv_leader + static_cast<uint32_t>(s) * 8u);
-        // next k-block's scales: issued after the fence so that it never waits for them
-        if (kb + 1 < KB) {
-#pragma unroll
-          for (int j = 0; j < (TNH + 15) / 16; ++j) {
-            const int r = r0 + 16 * j;
-            sc_next[j] = (r < TNH && b_row + r < args.n_out) ? srow[static_cast<size_t>(r) * KS + (kb + 1) * 2]
-                                                             : uint8_t(127);
-          }
+        if (lane == 0) {
+          mbar_arrive_cluster(conv_leader + static_cast<uint32_t>(s) * 8u);
+          mbar_arrive(&pempty[p]);
         }
         if (++s == STAGES) { s = 0; ph ^= 1u; }
+        if (++p == PS) { p = 0; pph ^= 1u; }
       }
     }
     if (!ok) {

@@ -59,11 +59,17 @@ cudaError_t combine_gather(const Launch& L, bool bf16, int64_t T, int D, int k, 
 cudaError_t combine_slots(const Launch& L, bool bf16, int64_t T, int D, int k, const void* ys, void* y);
 
 // The same two projections with MXFP4 expert weights, dequantised inside the GEMM mainloop.
+// The kernels read the E8M0 scales from a copy relaid as [E][ceil(K/64)][N][2]
+// (mx_scale_bytes each), written by mx_scale_relayout on the same stream.
+size_t mx_scale_bytes(int rows, int K, int E);
+cudaError_t mx_scale_relayout(const Launch& L, int D, int F, int E, const ExpertWeights& w, uint8_t* s_gate,
+                              uint8_t* s_up, uint8_t* s_down);
 cudaError_t expert_gateup_mxfp4(const Launch& L, int64_t R, int D, int F, int E, const void* x_perm,
-                                const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h);
+                                const int32_t* expert_off, const ExpertWeights& w, const uint8_t* s_gate2,
+                                const uint8_t* s_up2, float limit, float alpha, void* h);
 cudaError_t expert_down_mxfp4(const Launch& L, int64_t R, int D, int F, int E, const void* h,
-                              const int32_t* expert_off, const ExpertWeights& w, const int32_t* slot_of_row,
-                              const float* topk_w, void* out);
+                              const int32_t* expert_off, const ExpertWeights& w, const uint8_t* s_down2,
+                              const int32_t* slot_of_row, const float* topk_w, void* out);
 
 cudaError_t read_and_clear_device_error(int* bits);
 

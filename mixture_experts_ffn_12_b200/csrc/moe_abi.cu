@@ -57,8 +57,21 @@ bool check_T(int64_t T, int k) { return T >= 0 && T * k < (int64_t(1) << 31); }
 
 size_t elem_size(const moe_config_t* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
 
-// The expert GEMMs need no scratch (MXFP4 weights are dequantised in the mainloop).
-size_t ffn_ws_bytes(const moe_config_t*, int64_t) { return 0; }
+// Scratch of the expert GEMMs: none for dense weights; for MXFP4 the three scale
+// tensors relaid for TMA ([E][ceil(K/64)][N][2] each, 256-byte aligned regions).
+struct MxScaleRegions {
+  size_t gate, up, down, total;
+};
+MxScaleRegions mx_regions(const moe_config_t* c) {
+  const int D = c->hidden_size, F = c->intermediate_size, E = c->num_local_experts;
+  MxScaleRegions r{};
+  r.gate = 0;
+  r.up = align256(moe::mx_scale_bytes(F, D, E));
+  r.down = r.up + align256(moe::mx_scale_bytes(F, D, E));
+  r.total = r.down + align256(moe::mx_scale_bytes(D, F, E));
+  return r;
+}
+size_t ffn_ws_bytes(const moe_config_t* c, int64_t) { return c->wfmt == MOE_W_MXFP4 ? mx_regions(c).total : 0; }
 
 struct Layout {
   size_t ids, w, off, ros, sor, pscr, xperm, h, rpart, ys, ffn, total;
@@ -147,12 +160,17 @@ moe_status_t run_experts(const moe_config_t* c, const Launch& L, int64_t T, cons
   moe::ExpertWeights w = to_internal(wts);
   stage_mark(ST_GATEUP, true, L.stream);
   if (c->wfmt == MOE_W_MXFP4) {
-    if (moe::expert_gateup_mxfp4(L, R, D, F, E, x_perm, eoff, w, c->swiglu_limit, c->swiglu_alpha, h) !=
-        cudaSuccess)
+    const MxScaleRegions rg = mx_regions(c);
+    uint8_t* ws = static_cast<uint8_t*>(ffn_ws);
+    if (moe::mx_scale_relayout(L, D, F, E, w, ws + rg.gate, ws + rg.up, ws + rg.down) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (moe::expert_gateup_mxfp4(L, R, D, F, E, x_perm, eoff, w, ws + rg.gate, ws + rg.up, c->swiglu_limit,
+                                 c->swiglu_alpha, h) != cudaSuccess)
       return MOE_ERR_CUDA;
     stage_mark(ST_GATEUP, false, L.stream);
     stage_mark(ST_DOWN, true, L.stream);
-    const moe_status_t st = cuda_status(moe::expert_down_mxfp4(L, R, D, F, E, h, eoff, w, slot_of_row, topk_w, out));
+    const moe_status_t st =
+        cuda_status(moe::expert_down_mxfp4(L, R, D, F, E, h, eoff, w, ws + rg.down, slot_of_row, topk_w, out));
     stage_mark(ST_DOWN, false, L.stream);
     return st;
   }

@@ -91,7 +91,12 @@ def test_workspace_sizes(lib):
     assert lib.moe_workspace_size(ctypes.byref(c), -1) == _lib.SIZE_INVALID
     assert lib.moe_workspace_size(ctypes.byref(c), 1 << 30) == _lib.SIZE_INVALID   # T*k >= 2^31
     mx = cfg(wfmt=_lib.MOE_W_MXFP4)
-    assert lib.moe_expert_ffn_workspace_size(ctypes.byref(mx), 8) == 0     # dequantised in the mainloop
+    # MXFP4: the three scale tensors relaid as [E][ceil(K/64)][N][2], 256-byte aligned regions
+    E = 32
+    gu = -(-(E * (D // 64) * F * 2) // 256) * 256
+    dn = -(-(E * (F // 64) * D * 2) // 256) * 256
+    assert lib.moe_expert_ffn_workspace_size(ctypes.byref(mx), 8) == 2 * gu + dn
+    assert lib.moe_expert_ffn_workspace_size(ctypes.byref(mx), 4096) == 2 * gu + dn
 
 
 def test_rejections_launch_nothing(lib):
