@@ -19,12 +19,14 @@
 // written by mx_scale_relayout_kernel each call), because rows of K/32 bytes are
 // not a multiple of 16 bytes and cannot be described to TMA as they are stored.
 //
-// Roles (480 threads per CTA):
+// Roles (608 threads per CTA):
 //   warp 0      activation producer (TMA, both CTAs, bytes counted on the leader)
 //   warp 1      TMEM; the leader's lane 0 issues the pair MMAs
 //   warps 2-5   epilogue (this CTA's 128 accumulator rows)
 //   warp 6      packed-weight producer (TMA into the packed ring, this CTA)
-//   warps 7-14  converters (two per SM sub-partition, so one's latency hides the other's)
+//   warps 7-18  converters, in three groups of four warps: group g decodes the K steps
+//               j with j % 3 == g (every row of the step), so three steps are decoded
+//               at once and a step's decode latency is hidden behind the other two
 #pragma once
 
 #include "grouped_gemm_pair.cuh"
@@ -32,8 +34,9 @@
 namespace moe {
 
 constexpr int kMxConvWarp0 = 7;     // first converter warp
-constexpr int kMxConvWarps = 8;
-constexpr int kMxThreads = (kMxConvWarp0 + kMxConvWarps) * 32;
+constexpr int kMxConvGroups = 3;    // K steps decoded concurrently
+constexpr int kMxGroupWarps = 4;    // warps per group (one per SM sub-partition)
+constexpr int kMxThreads = (kMxConvWarp0 + kMxConvGroups * kMxGroupWarps) * 32;
 constexpr int kMxPackSlots = 16;    // depth of the packed-weight ring
 
 template <int TNH>
@@ -141,9 +144,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
   uint8_t* pring = smem + STAGES * LY::STAGE_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(pring + PS * LY::SLOT_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* conv = empty + STAGES;         // both CTAs' weight halves decoded (leader, 2 x kMxConvWarps arrivals)
+  uint64_t* conv = empty + STAGES;         // both CTAs' weight halves decoded (leader, one group of each CTA)
   uint64_t* pfull = conv + STAGES;         // packed slot landed (local, TMA)
-  uint64_t* pempty = pfull + PS;           // packed slot read by the local converter warps
+  uint64_t* pempty = pfull + PS;           // packed slot read by the local group that decoded it
   uint64_t* tfull = pempty + PS;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
@@ -167,11 +170,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&conv[s], 2 * kMxConvWarps);
+      mbar_init(&conv[s], 2 * kMxGroupWarps);
     }
     for (int p = 0; p < PS; ++p) {
       mbar_init(&pfull[p], 1);
-      mbar_init(&pempty[p], kMxConvWarps);
+      mbar_init(&pempty[p], kMxGroupWarps);
     }
     mbar_init(&tfull[0], 1);
     mbar_init(&tfull[1], 1);
@@ -368,39 +371,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ converters (both CTAs)
-    constexpr int kRowStep = kMxConvWarps * 4;           // rows r0, r0 + kRowStep, ...
-    const int ct = threadIdx.x - kMxConvWarp0 * 32;      // 0 .. 32 * kMxConvWarps - 1
+    const int cw = warp - kMxConvWarp0;                  // 0 .. groups * group warps - 1
+    const int grp = cw / kMxGroupWarps;
+    const int ct = (cw % kMxGroupWarps) * 32 + lane;     // 0..127 within the group
     const uint32_t conv_leader = mapa_shared(smem_u32(conv), 0);
     const int c = ct & 7;                                // 4-byte chunk of a 32-byte packed row (8 codes)
-    const int r0 = ct >> 3;
-    int s = 0, p = 0;
-    uint32_t ph = 0, pph = 0;
+    const int r0 = ct >> 3;                              // rows r0, r0 + 16, ...
+    // this cluster's K steps, numbered across its tiles like the producers walk them
+    const int my_tiles = cluster < total ? (total - cluster + nclusters - 1) / nclusters : 0;
+    const int steps = my_tiles * KB;
     bool ok = true;
-    for (int i = cluster; ok && i < total; i += nclusters) {
-      for (int kb = 0; kb < KB; ++kb) {
-        // packed slot landed, and the MMA is done with this stage's weight tile
-        if (!__all_sync(0xffffffffu, mbar_wait(&pfull[p], pph, abort_flag, lim))) { ok = false; break; }
-        if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim))) { ok = false; break; }
-        const uint8_t* sp = pring + p * LY::SLOT_BYTES;
-        const uint8_t* ss = sp + LY::P_BYTES;
-        uint8_t* sb = smem + s * LY::STAGE_BYTES + LY::A_BYTES;
+    for (int j = grp; ok && j < steps; j += kMxConvGroups) {
+      const int s = j % STAGES, p = j % PS;
+      const uint32_t ph = static_cast<uint32_t>(j / STAGES) & 1u, pph = static_cast<uint32_t>(j / PS) & 1u;
+      // packed slot landed, and the MMA is done with this stage's weight tile
+      if (!__all_sync(0xffffffffu, mbar_wait(&pfull[p], pph, abort_flag, lim))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim))) { ok = false; break; }
+      const uint8_t* sp = pring + p * LY::SLOT_BYTES;
+      const uint8_t* ss = sp + LY::P_BYTES;
+      uint8_t* sb = smem + s * LY::STAGE_BYTES + LY::A_BYTES;
 #pragma unroll
-        for (int j = 0; j < (TNH + kRowStep - 1) / kRowStep; ++j) {
-          const int r = r0 + kRowStep * j;
-          if (r < TNH) {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(sp + r * 32 + c * 4);
-            const uint4 v = mxfp4_decode8(w, e8m0_to_bf16x2(ss[r * 2 + (c >> 2)]));
-            *reinterpret_cast<uint4*>(sb + r * kRowBytes + ((c ^ (r & 7)) << 4)) = v;
-          }
+      for (int q = 0; q < (TNH + 15) / 16; ++q) {
+        const int r = r0 + 16 * q;
+        if (r < TNH) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(sp + r * 32 + c * 4);
+          const uint4 v = mxfp4_decode8(w, e8m0_to_bf16x2(ss[r * 2 + (c >> 2)]));
+          *reinterpret_cast<uint4*>(sb + r * kRowBytes + ((c ^ (r & 7)) << 4)) = v;
         }
-        fence_proxy_async_smem();     // generic-proxy stores -> visible to the tensor core
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_cluster(conv_leader + static_cast<uint32_t>(s) * 8u);
-          mbar_arrive(&pempty[p]);
-        }
-        if (++s == STAGES) { s = 0; ph ^= 1u; }
-        if (++p == PS) { p = 0; pph ^= 1u; }
+      }
+      fence_proxy_async_smem();     // generic-proxy stores -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_cluster(conv_leader + static_cast<uint32_t>(s) * 8u);
+        mbar_arrive(&pempty[p]);
       }
     }
     if (!ok) {
