@@ -49,6 +49,7 @@ def parse_args():
     p.add_argument("--workload", default="gptoss20b_prefill", choices=sorted(W.SPECS))
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-decode", action="store_true", help="skip the decode-regime sweep")
+    p.add_argument("--no-mxfp4", action="store_true", help="skip the MXFP4-weight layer")
     return p.parse_args()
 
 
@@ -301,6 +302,11 @@ def run_ours(args, rank, world, local_rank):
     ms_e2e = max_over_ranks(e0.elapsed_time(e1))
 
     decode = decode_sweep(api, moe, spec, layer, dev, stream, max(20, K // 4)) if not args.no_decode else None
+    mx = None
+    if not args.no_mxfp4 and world == 1 and spec.wfmt == "dense" and spec.dtype == "bf16":
+        del d, moe
+        torch.cuda.empty_cache()
+        mx = mxfp4_sweep(api, dev, stream, max(10, K // 10))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -337,6 +343,8 @@ def run_ours(args, rank, world, local_rank):
         }
         if decode is not None:
             line["decode"] = decode
+        if mx is not None:
+            line["mxfp4"] = mx
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
@@ -380,6 +388,49 @@ def decode_sweep(api, moe, spec, layer, dev, stream, steps):
         out[f"T{T}"] = {"us_per_step": us, "experts_touched": touched, "weight_bytes": nbytes, "GB/s": gbs,
                         "hbm_frac": gbs / peaks["hbm_gbs"], "tokens/s": T / (us * 1e-6)}
     return out
+
+
+def mxfp4_sweep(api, dev, stream, steps):
+    """The same layer with MXFP4 expert weights (GPT-OSS-20B shape, T = 8192): per-step time,
+    stage times and the gate/up GEMM's TFLOP/s.  The MXFP4 weights are decoded to bf16 inside
+    the GEMM mainloop; the FLOPs counted are the bf16 MMA work (4*R*D*F for gate/up)."""
+    import torch
+    from mixture_experts_ffn_12_b200 import _lib
+    spec = W.GPTOSS20B_MXFP4
+    peaks = measured_peaks()
+    layer = W.make_layer(spec, seed=0)
+    d = api.upload_layer(layer, dev)
+    moe = api.MoELayer(api.config_from_spec(spec), d["w_router"], d["b_router"], api.expert_weights_from(d))
+    x = d["x"]
+    y = torch.empty_like(x)
+    for _ in range(3):
+        moe(x, y=y)
+    torch.cuda.synchronize()
+    lib = _lib.load()
+    n = len(STAGES)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        hs = [ctypes_ptr(e.cuda_event) for e in ev[i]]
+        lib.moe_set_stage_events((_lib.ctypes.c_void_p * n)(*hs[:n]), (_lib.ctypes.c_void_p * n)(*hs[n:]), n)
+        moe(x, y=y)
+    b.record(stream)
+    lib.moe_set_stage_events(None, None, 0)
+    torch.cuda.synchronize()
+    if api.last_device_error() != 0:
+        raise RuntimeError("device error word set during the MXFP4 steps")
+    us = 1e3 * a.elapsed_time(b) / steps
+    stage = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][n + j]) for i in range(steps)) * 1e3
+             for j, name in enumerate(STAGES)}
+    gu_tf = 4.0 * spec.R * spec.D * spec.F / (stage["gateup_swiglu_gemm"] * 1e-6) / 1e12
+    return {"workload": spec.name, "T": spec.T, "us_per_step": us, "tokens/s": spec.T / (us * 1e-6),
+            "stage_us": stage, "gateup_tflops": gu_tf, "gateup_frac": gu_tf / peaks["bf16_tflops"],
+            "weight_bytes": 3 * spec.E * spec.D * spec.F // 2 + 3 * spec.E * spec.D * spec.F // 32}
 
 
 def reduce_max(v: float, device) -> float:

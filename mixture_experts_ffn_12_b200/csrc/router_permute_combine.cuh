@@ -30,32 +30,48 @@ namespace moe {
 // ---------------------------------------------------------------------------
 constexpr int kRouterWarps = 32;   // one block per token: a warp per expert for E <= 32
 constexpr int kRouterSplits = 4;   // K ranges of the tensor-core router inside the fused layer
+constexpr int kRouterMaxChunks = 1024;   // x row staged in shared memory: D * elem <= 16 KB
+
+// Dot product of a row of x (staged in shared memory, or in global memory) with a weight row in global
+// memory; lanes stride over 16-byte chunks.  The weight loads of a batch are all
+// issued before any is used, so a row costs ceil(chunks / (32 * kDotBatch)) memory
+// round trips instead of one per chunk a lane handles.
+constexpr int kDotBatch = 6;
 
 template <typename T>
-__device__ __forceinline__ float dot_row16(const T* a, const T* b, int D, int lane) {
-  // 16-byte chunks of both rows, lanes strided over the chunks
+__device__ __forceinline__ float dot_row16(const uint4* xs, const T* b, int D, int lane) {
   constexpr int EPC = 16 / sizeof(T);
   const int nchunk = D / EPC;
-  const uint4* pa = reinterpret_cast<const uint4*>(a);
   const uint4* pb = reinterpret_cast<const uint4*>(b);
   float acc = 0.0f;
-#pragma unroll 6
-  for (int c = lane; c < nchunk; c += 32) {
-    const uint4 ua = pa[c], ub = pb[c];
-    if constexpr (sizeof(T) == 4) {
-      const float* fa = reinterpret_cast<const float*>(&ua);
-      const float* fb = reinterpret_cast<const float*>(&ub);
+  for (int c0 = lane; c0 < nchunk; c0 += 32 * kDotBatch) {
+    uint4 wv[kDotBatch];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc = fmaf(fa[i], fb[i], acc);
-    } else {
-      const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&ua);
-      const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&ub);
+    for (int u = 0; u < kDotBatch; ++u) {
+      const int c = c0 + 32 * u;
+      wv[u] = c < nchunk ? pb[c] : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 fa = __bfloat1622float2(ha[i]);
-        const float2 fb = __bfloat1622float2(hb[i]);
-        acc = fmaf(fa.x, fb.x, acc);
-        acc = fmaf(fa.y, fb.y, acc);
+    for (int u = 0; u < kDotBatch; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nchunk) {
+        const uint4 ua = xs[c];
+        if constexpr (sizeof(T) == 4) {
+          const float* fa = reinterpret_cast<const float*>(&ua);
+          const float* fb = reinterpret_cast<const float*>(&wv[u]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc = fmaf(fa[i], fb[i], acc);
+        } else {
+          const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&ua);
+          const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&wv[u]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 fa = __bfloat1622float2(ha[i]);
+            const float2 fb = __bfloat1622float2(hb[i]);
+            acc = fmaf(fa.x, fb.x, acc);
+            acc = fmaf(fa.y, fb.y, acc);
+          }
+        }
       }
     }
   }
@@ -151,11 +167,17 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
     router_simt_kernel(const T* __restrict__ x, const T* __restrict__ wr, const T* __restrict__ br, int D, int E,
                        int k, int32_t* __restrict__ ids, float* __restrict__ wout) {
   __shared__ float logits[256];
+  __shared__ uint4 xs[kRouterMaxChunks];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const T* xr = x + static_cast<size_t>(t) * D;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * D);
+  const int nchunk = D * static_cast<int>(sizeof(T)) / 16;
+  const bool staged = nchunk <= kRouterMaxChunks;        // else the row is read from global memory
+  if (staged)
+    for (int c = threadIdx.x; c < nchunk; c += blockDim.x) xs[c] = xr[c];
+  __syncthreads();
   for (int e = warp; e < E; e += kRouterWarps) {
-    const float l = dot_row16<T>(xr, wr + static_cast<size_t>(e) * D, D, lane);
+    const float l = dot_row16<T>(staged ? xs : xr, wr + static_cast<size_t>(e) * D, D, lane);
     if (lane == 0) logits[e] = l + to_f32<T>(br[e]);
   }
   __syncthreads();
@@ -401,12 +423,26 @@ __global__ void __launch_bounds__(kChunk) permute_small_kernel(const int32_t* __
   }
   __syncthreads();
   if (x == nullptr) return;
-  for (int r = warp; r < R; r += kChunkWarps) {
-    const int src = sor[r] / k;
-    if (src < 0 || src >= T) continue;
-    const uint4* a = x + static_cast<size_t>(src) * vec_per_row;
-    uint4* b = x_perm + static_cast<size_t>(r) * vec_per_row;
-    for (int v = lane; v < vec_per_row; v += 32) b[v] = a[v];
+  // (row, chunk) pairs spread over the block; each thread issues kCopyBatch loads before storing
+  constexpr int kCopyBatch = 16;
+  const int n = R * vec_per_row;
+  for (int i0 = threadIdx.x; i0 < n; i0 += kChunk * kCopyBatch) {
+    uint4 v[kCopyBatch];
+#pragma unroll
+    for (int u = 0; u < kCopyBatch; ++u) {
+      const int i = i0 + u * kChunk;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < n) {
+        const int r = i / vec_per_row;
+        const int src = sor[r] / k;
+        if (src >= 0 && src < T) v[u] = x[static_cast<size_t>(src) * vec_per_row + (i - r * vec_per_row)];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyBatch; ++u) {
+      const int i = i0 + u * kChunk;
+      if (i < n) x_perm[i] = v[u];
+    }
   }
 }
 
