@@ -220,7 +220,8 @@ MOE_API void moe_set_stage_events(void* const* starts, void* const* stops, int32
 
 /* Tuning knob for the bf16 expert GEMMs of every later call in this process:
  * 0 = choose by size (default: the weight-stationary decode kernel while the
- * experts average at most 16 routed rows, single-CTA 128-row tiles otherwise),
+ * experts average at most 16 routed rows; otherwise single-CTA 128-row tiles for
+ * gate/up and CTA-pair tiles for down),
  * 1 = single-CTA tiles, 2 = CTA-pair tiles (256 rows), 3 = decode kernel,
  * 4 = CTA pairs with the expert weights as the MMA's M operand (tokens in N).
  * Results are the same up to fp32 accumulation order.  MOE_ERR_INVALID_ARG for

@@ -196,13 +196,15 @@ inline std::atomic<int> g_gemm_variant{0};
 enum GemmKind { GK_SINGLE = 1, GK_PAIR = 2, GK_DECODE = 3, GK_WM_PAIR = 4 };
 
 // By default: the decode kernel while experts average at most 16 rows (the
-// layer is a weight stream), single-CTA 128-row tiles otherwise.
-static GemmKind gemm_kind(int64_t R, int E) {
+// layer is a weight stream); otherwise single-CTA 128-row tiles for gate/up and
+// CTA pairs for down (measured fastest for each on the GPT-OSS shapes).
+static GemmKind gemm_kind(int64_t R, int E, bool down = false) {
   const int v = g_gemm_variant.load();
   if (v >= 1 && v <= 4) return static_cast<GemmKind>(v);
-  return R <= int64_t(16) * E ? GK_DECODE : GK_SINGLE;
+  if (R <= int64_t(16) * E) return GK_DECODE;
+  return down ? GK_PAIR : GK_SINGLE;
 }
-static bool use_pair(int64_t R, int E) { return gemm_kind(R, E) == GK_PAIR; }
+static bool use_pair(int64_t R, int E, bool down = false) { return gemm_kind(R, E, down) == GK_PAIR; }
 
 constexpr int kDecTok = 32;
 
@@ -473,7 +475,7 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
   a.ldo = D;
   a.slot_of_row = slot_of_row;
   a.topk_w = topk_w;
-  if (gemm_kind(R, E) == GK_DECODE) {
+  if (gemm_kind(R, E, true) == GK_DECODE) {
     CUtensorMap wd, th;
     if ((e = make_tmap(&wd, w.w_down, false, F, D, E, 128)) != cudaSuccess) return e;
     if ((e = make_tmap(&th, h, false, F, R, 0, kDecTok)) != cudaSuccess) return e;
@@ -481,7 +483,7 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
     if (slot_of_row != nullptr) return launch_decode<EPI_BIAS_WSCATTER>(L, wd, wd, th, a, units);
     return launch_decode<EPI_BIAS>(L, wd, wd, th, a, units);
   }
-  if (gemm_kind(R, E) == GK_WM_PAIR) {
+  if (gemm_kind(R, E, true) == GK_WM_PAIR) {
     CUtensorMap wd, th16;
     if ((e = make_tmap(&wd, w.w_down, false, F, D, E, 128)) != cudaSuccess) return e;
     if ((e = make_tmap(&th16, h, false, F, R, 0, 16)) != cudaSuccess) return e;
@@ -489,7 +491,7 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
     if (slot_of_row != nullptr) return launch_wm_pair<EPI_BIAS_WSCATTER>(L, wd, wd, ta, th16, a, units);
     return launch_wm_pair<EPI_BIAS>(L, wd, wd, ta, th16, a, units);
   }
-  const bool pair = use_pair(R, E);
+  const bool pair = use_pair(R, E, true);
   if ((e = make_tmap(&tb, w.w_down, !bf16, F, D, E, pair ? kTNHalf : kTNDown)) != cudaSuccess) return e;
   if (pair) {
     const int64_t ptiles = ((R + kPairBM - 1) / kPairBM + E) * ((D + 2 * kTNHalf - 1) / (2 * kTNHalf));
