@@ -21,7 +21,8 @@
 
 namespace moe {
 
-constexpr int kDecStages = 10;
+constexpr int kDecStages = 10;       // one CTA per SM
+constexpr int kDecStagesDual = 5;    // two CTAs per SM
 constexpr int kDecTmemCols = 64;   // two accumulators of NTOK = 32 columns
 
 template <int NTOK>
@@ -30,9 +31,11 @@ struct DecLayout {
   static constexpr int X_BYTES = NTOK * kRowBytes;
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
   static constexpr int UP_BYTES = 64 * NTOK * 4;      // up values handed to the gate warps
-  static constexpr int EXTRA = 1024 + 4096;
+  static constexpr int EXTRA = 1024 + 2560;   // alignment slack; barriers, unit and group offsets (2.3 KB)
   static constexpr int smem_bytes(int stages) { return stages * STAGE_BYTES + UP_BYTES + EXTRA; }
   static_assert(NTOK % 16 == 0 && NTOK <= 256, "MMA N");
+  static_assert(2 * (STAGE_BYTES * kDecStagesDual + UP_BYTES + EXTRA + 1024) <= 233472,
+                "two CTAs per SM (plus 1 KB reserved each) fit the 228 KB of shared memory");
 };
 
 struct UnitInfo {

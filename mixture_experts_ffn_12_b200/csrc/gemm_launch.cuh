@@ -208,12 +208,11 @@ static bool use_pair(int64_t R, int E, bool down = false) { return gemm_kind(R, 
 
 constexpr int kDecTok = 32;
 
-template <int EPI>
-static cudaError_t launch_decode(const Launch& L, const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x,
-                                 const GemmArgs& args, int64_t max_units) {
-  if (max_units <= 0) return cudaSuccess;
-  auto kern = decode_gemm_kernel<EPI, kDecTok, kDecStages>;
-  constexpr int smem = DecLayout<kDecTok>::smem_bytes(kDecStages);
+template <int EPI, int STAGES>
+static cudaError_t launch_decode_st(const Launch& L, const CUtensorMap& w0, const CUtensorMap& w1,
+                                    const CUtensorMap& x, const GemmArgs& args, int grid) {
+  auto kern = decode_gemm_kernel<EPI, kDecTok, STAGES>;
+  constexpr int smem = DecLayout<kDecTok>::smem_bytes(STAGES);
   static_assert(smem <= 232448, "shared memory budget");
   int dev = 0;
   cudaGetDevice(&dev);
@@ -227,10 +226,23 @@ static cudaError_t launch_decode(const Launch& L, const CUtensorMap& w0, const C
       if (dev < 64) configured |= uint64_t(1) << dev;
     }
   }
-  const int grid = static_cast<int>(std::min<int64_t>(max_units, L.num_sms));
   kern<<<grid, kGemmThreads, smem, L.stream>>>(w0, w1, x, args);
   count_launch();
   return cudaGetLastError();
+}
+
+// Up to one unit per SM: one CTA per SM with the deep ring.  More units than SMs:
+// two CTAs per SM with half the ring each, so every unit of a short list (T = 1
+// gate/up: 4 experts x 45 feature blocks = 180 units) streams at once instead of
+// a second partial wave.
+template <int EPI>
+static cudaError_t launch_decode(const Launch& L, const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x,
+                                 const GemmArgs& args, int64_t max_units) {
+  if (max_units <= 0) return cudaSuccess;
+  if (max_units <= L.num_sms)
+    return launch_decode_st<EPI, kDecStages>(L, w0, w1, x, args, static_cast<int>(max_units));
+  const int grid = static_cast<int>(std::min<int64_t>(max_units, int64_t(2) * L.num_sms));
+  return launch_decode_st<EPI, kDecStagesDual>(L, w0, w1, x, args, grid);
 }
 
 static GemmArgs base_args(const Launch& L) {
