@@ -68,7 +68,7 @@ struct GemmArgs {
   const uint8_t* scale0;       // MXFP4: E8M0 scales of B0 / B1, [G, n_out, k_dim / 32]
   const uint8_t* scale1;
   int k_splits;                // EPI_PARTIAL: K ranges; column block index = K range
-  float* partial;              // EPI_PARTIAL: [k_splits, m_total, n_out] fp32
+  float* partial;              // EPI_PARTIAL: [k_splits, n_out, m_total] fp32
 };
 
 constexpr int kBM = 128;           // rows per tile (MMA M)
@@ -236,9 +236,11 @@ __device__ __forceinline__ void epi_topk(uint32_t tbase, int row, bool rvalid, c
   }
 }
 
+// Partial logits go to partial[split][e][row] (expert-major), so for each column
+// the 32 rows of a warp store 128 contiguous bytes.
 __device__ __forceinline__ void epi_partial(uint32_t tbase, int row, bool rvalid, const TileInfo& ti,
                                             const GemmArgs& a, int split) {
-  float* out = a.partial + (static_cast<size_t>(split) * a.m_total + row) * a.n_out;
+  float* out = a.partial + static_cast<size_t>(split) * a.n_out * a.m_total + row;
 #pragma unroll 1
   for (int c = 0; c < a.mma_n; c += 8) {
     float v[8];
@@ -247,7 +249,7 @@ __device__ __forceinline__ void epi_partial(uint32_t tbase, int row, bool rvalid
     if (rvalid) {
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (c + j < a.n_out) out[c + j] = v[j];
+        if (c + j < a.n_out) out[static_cast<size_t>(c + j) * a.m_total] = v[j];
     }
   }
 }

@@ -127,39 +127,111 @@ __device__ __forceinline__ void warp_topk_softmax(float (&v)[8], int lane, int E
   }
 }
 
-// Fused-layer router tail: sum of the K-range partial logits + router bias, then
-// top-k and softmax.  One warp per token.
-template <typename T, int SPLITS>
+// Fused-layer router tail: sum of the K-range partial logits (partial[split][e][t])
+// + router bias, top-k and the softmax over the k selected.  P threads per token
+// (P = power of two >= E / 32), each scanning up to 32 experts: thread (part, t)
+// with t fastest in the block, so each expert's loads are coalesced across tokens.
+// Each thread keeps a running top-k of its experts in index order (strict '>'
+// keeps the lower index first on ties); part 0 merges the P lists through shared
+// memory, taking lower parts first on ties, which keeps the global order.
+template <typename T, int SPLITS, int P>
 __global__ void __launch_bounds__(256) router_topk_partials_kernel(const float* __restrict__ partial,
                                                                    const T* __restrict__ br, int Tn, int E, int k,
                                                                    int32_t* __restrict__ ids,
                                                                    float* __restrict__ wout) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= Tn) return;
-  // all loads first (they are independent), then the sums in split order
-  float p[8][SPLITS];
+  constexpr int TPB = 256 / P;                       // tokens per block
+  __shared__ float bias[256];
+  __shared__ float lv[P][8][TPB];
+  __shared__ int li[P][8][TPB];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) bias[e] = to_f32<T>(br[e]);
+  __syncthreads();
+  const int part = threadIdx.x / TPB, tl = threadIdx.x % TPB;
+  const int t = blockIdx.x * TPB + tl;
+  const bool tv_ok = t < Tn;
+  float tv[8];
+  int tix[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
+  for (int j = 0; j < 8; ++j) { tv[j] = -INFINITY; tix[j] = 0x7fffffff; }
+  const size_t plane = static_cast<size_t>(E) * Tn;
+  const int e_begin = part * 32, e_end = min(E, e_begin + 32);
+  if (tv_ok) {
+#pragma unroll 1
+    for (int e0 = e_begin; e0 < e_end; e0 += 8) {
+      float p[8][SPLITS];
 #pragma unroll
-    for (int sp = 0; sp < SPLITS; ++sp)
-      p[i][sp] = e < E ? __ldcg(partial + (static_cast<size_t>(sp) * Tn + t) * E + e) : 0.0f;
-  }
-  float v[8];
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    float acc = -INFINITY;
-    if (e < E) {
-      acc = p[i][0];
+        for (int sp = 0; sp < SPLITS; ++sp)
+          p[i][sp] = e0 + i < e_end ? __ldcg(partial + sp * plane + static_cast<size_t>(e0 + i) * Tn + t) : 0.0f;
 #pragma unroll
-      for (int sp = 1; sp < SPLITS; ++sp) acc += p[i][sp];
-      acc += to_f32<T>(br[e]);
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i;
+        if (e >= e_end) break;
+        float cv = p[i][0];
+#pragma unroll
+        for (int sp = 1; sp < SPLITS; ++sp) cv += p[i][sp];
+        cv += bias[e];
+        int ci = e;
+        if (cv > tv[7]) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const bool gt = cv > tv[q];
+            const float tq = tv[q];
+            const int iq = tix[q];
+            tv[q] = gt ? cv : tq;
+            tix[q] = gt ? ci : iq;
+            cv = gt ? tq : cv;
+            ci = gt ? iq : ci;
+          }
+        }
+      }
     }
-    v[i] = acc;
   }
-  warp_topk_softmax(v, lane, E, k, ids + static_cast<size_t>(t) * k, wout + static_cast<size_t>(t) * k);
+  if constexpr (P > 1) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      lv[part][j][tl] = tv[j];
+      li[part][j][tl] = tix[j];
+    }
+    __syncthreads();
+    if (part != 0) return;
+    // merge parts 1..P-1 into part 0's list; a candidate displaces only on '>', and
+    // parts come in increasing expert order, so ties keep the lower index first
+#pragma unroll 1
+    for (int q2 = 1; q2 < P; ++q2) {
+#pragma unroll
+      for (int j2 = 0; j2 < 8; ++j2) {
+        float cv = lv[q2][j2][tl];
+        int ci = li[q2][j2][tl];
+        if (cv > tv[7]) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const bool gt = cv > tv[q];
+            const float tq = tv[q];
+            const int iq = tix[q];
+            tv[q] = gt ? cv : tq;
+            tix[q] = gt ? ci : iq;
+            cv = gt ? tq : cv;
+            ci = gt ? iq : ci;
+          }
+        }
+      }
+    }
+  }
+  if (!tv_ok) return;
+  float z = 0.0f, ex[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    ex[j] = j < k ? expf(tv[j] - tv[0]) : 0.0f;
+    z += ex[j];
+  }
+  const float inv = 1.0f / z;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < k) {
+      ids[static_cast<size_t>(t) * k + j] = tix[j];
+      wout[static_cast<size_t>(t) * k + j] = ex[j] * inv;
+    }
 }
 
 template <typename T>
@@ -208,8 +280,20 @@ cudaError_t router_topk(const Launch& L, bool bf16, int64_t T, int D, int E, int
     // K split over kRouterSplits ranges so that more CTAs stream x, then sum + top-k
     cudaError_t e = router_tc_partial(L, T, D, E, kRouterSplits, x, w_router, partial);
     if (e != cudaSuccess) return e;
-    router_topk_partials_kernel<__nv_bfloat16, kRouterSplits><<<static_cast<unsigned>((T + 7) / 8), 256, 0, L.stream>>>(
-        partial, static_cast<const __nv_bfloat16*>(b_router), static_cast<int>(T), E, k, ids, w);
+    const __nv_bfloat16* br = static_cast<const __nv_bfloat16*>(b_router);
+    const int Ti = static_cast<int>(T);
+    if (E <= 32)
+      router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 1><<<(Ti + 255) / 256, 256, 0, L.stream>>>(
+          partial, br, Ti, E, k, ids, w);
+    else if (E <= 64)
+      router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 2><<<(Ti + 127) / 128, 256, 0, L.stream>>>(
+          partial, br, Ti, E, k, ids, w);
+    else if (E <= 128)
+      router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 4><<<(Ti + 63) / 64, 256, 0, L.stream>>>(
+          partial, br, Ti, E, k, ids, w);
+    else
+      router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 8><<<(Ti + 31) / 32, 256, 0, L.stream>>>(
+          partial, br, Ti, E, k, ids, w);
     count_launch();
     return cudaGetLastError();
   }
