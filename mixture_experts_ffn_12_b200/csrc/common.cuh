@@ -12,6 +12,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "this library targets sm_100a (B200) only"
 #endif
@@ -29,6 +31,34 @@ enum : int {
 __device__ int g_device_error = 0;
 
 __device__ __forceinline__ void flag_error(int bits) { atomicOr(&g_device_error, bits); }
+
+// Programmatic dependent launch.  Every kernel of the library starts with this:
+// it lets the next kernel on the stream be scheduled (its CTAs then sit in their
+// own wait, so launch latency and CTA start-up overlap this kernel's tail) and
+// waits until the previous kernel has completed and its writes are visible.  A
+// kernel launched without the attribute passes straight through.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Host: launch `kern` on `stream` with programmatic stream serialization allowed.
+// Errors are left for cudaGetLastError, as with <<<>>>.
+template <typename... KArgs, typename... Args>
+inline void pdl_launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // --------------------------------------------------------------------------
 // basic

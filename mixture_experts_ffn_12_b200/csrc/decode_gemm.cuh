@@ -68,6 +68,7 @@ template <int EPI, int NTOK, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
                        const __grid_constant__ CUtensorMap tmX, const GemmArgs args) {
+  pdl_enter();
   using T = __nv_bfloat16;
   using LY = DecLayout<NTOK>;
   constexpr int BK = kRowBytes / 2;

@@ -105,7 +105,7 @@ static cudaError_t launch(const Launch& L, const CUtensorMap& a, const CUtensorM
     }
   }
   const int grid = static_cast<int>(std::min<int64_t>(max_tiles, L.num_sms));
-  kern<<<grid, kGemmThreads, smem, L.stream>>>(a, b0, b1, args);
+  pdl_launch(kern, dim3(grid), dim3(kGemmThreads), smem, L.stream, a, b0, b1, args);
   count_launch();
   return cudaGetLastError();
 }
@@ -131,7 +131,7 @@ static cudaError_t launch_pair(const Launch& L, const CUtensorMap& a, const CUte
     }
   }
   const int clusters = static_cast<int>(std::min<int64_t>(max_tiles, L.num_sms / 2));
-  kern<<<2 * clusters, kGemmThreads, smem, L.stream>>>(a, b0, b1, args);
+  pdl_launch(kern, dim3(2 * clusters), dim3(kGemmThreads), smem, L.stream, a, b0, b1, args);
   count_launch();
   return cudaGetLastError();
 }
@@ -157,7 +157,7 @@ static cudaError_t launch_pair_mx(const Launch& L, const CUtensorMap& a, const C
     }
   }
   const int clusters = static_cast<int>(std::min<int64_t>(max_tiles, L.num_sms / 2));
-  kern<<<2 * clusters, kMxThreads, smem, L.stream>>>(a, p0, p1, s0, s1, args);
+  pdl_launch(kern, dim3(2 * clusters), dim3(kMxThreads), smem, L.stream, a, p0, p1, s0, s1, args);
   count_launch();
   return cudaGetLastError();
 }
@@ -183,7 +183,7 @@ static cudaError_t launch_wm_pair(const Launch& L, const CUtensorMap& w0, const 
     }
   }
   const int clusters = static_cast<int>(std::min<int64_t>(max_units, L.num_sms / 2));
-  kern<<<2 * clusters, kGemmThreads, smem, L.stream>>>(w0, w1, x, x16, args);
+  pdl_launch(kern, dim3(2 * clusters), dim3(kGemmThreads), smem, L.stream, w0, w1, x, x16, args);
   count_launch();
   return cudaGetLastError();
 }
@@ -226,7 +226,7 @@ static cudaError_t launch_decode_st(const Launch& L, const CUtensorMap& w0, cons
       if (dev < 64) configured |= uint64_t(1) << dev;
     }
   }
-  kern<<<grid, kGemmThreads, smem, L.stream>>>(w0, w1, x, args);
+  pdl_launch(kern, dim3(grid), dim3(kGemmThreads), smem, L.stream, w0, w1, x, args);
   count_launch();
   return cudaGetLastError();
 }
@@ -324,7 +324,7 @@ cudaError_t mx_scale_relayout(const Launch& L, int D, int F, int E, const Expert
   job.groups = E;
   const int64_t most = std::max(mx_scale_bytes(F, D, E), mx_scale_bytes(D, F, E)) / 2;
   const dim3 grid(static_cast<unsigned>(std::min<int64_t>((most + 255) / 256, int64_t(8) * L.num_sms)), 3);
-  mx_scale_relayout_kernel<<<grid, 256, 0, L.stream>>>(job);
+  pdl_launch(mx_scale_relayout_kernel, dim3(grid), dim3(256), 0, L.stream, job);
   count_launch();
   return cudaGetLastError();
 }
@@ -401,7 +401,7 @@ cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, i
     a.out = h;
     a.ldo = F;
     const dim3 grid((F + kSimtBN - 1) / kSimtBN, static_cast<unsigned>((R + kSimtBM - 1) / kSimtBM + E));
-    simt_grouped_gemm_f32<EPI_SWIGLU><<<grid, 256, 0, L.stream>>>(
+    pdl_launch(simt_grouped_gemm_f32<EPI_SWIGLU>, dim3(grid), dim3(256), 0, L.stream, 
         static_cast<const float*>(x_perm), static_cast<const float*>(w.w_gate), static_cast<const float*>(w.w_up), a);
     count_launch();
     return cudaGetLastError();
@@ -465,10 +465,10 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
     a.topk_w = topk_w;
     const dim3 grid((D + kSimtBN - 1) / kSimtBN, static_cast<unsigned>((R + kSimtBM - 1) / kSimtBM + E));
     if (slot_of_row != nullptr)
-      simt_grouped_gemm_f32<EPI_BIAS_WSCATTER><<<grid, 256, 0, L.stream>>>(
+      pdl_launch(simt_grouped_gemm_f32<EPI_BIAS_WSCATTER>, dim3(grid), dim3(256), 0, L.stream, 
           static_cast<const float*>(h), static_cast<const float*>(w.w_down), nullptr, a);
     else
-      simt_grouped_gemm_f32<EPI_BIAS><<<grid, 256, 0, L.stream>>>(static_cast<const float*>(h),
+      pdl_launch(simt_grouped_gemm_f32<EPI_BIAS>, dim3(grid), dim3(256), 0, L.stream, static_cast<const float*>(h),
                                                                   static_cast<const float*>(w.w_down), nullptr, a);
     count_launch();
     return cudaGetLastError();

@@ -261,6 +261,7 @@ template <typename T, int TN, int NB, int EPI, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const GemmArgs args) {
+  pdl_enter();
   constexpr bool kTF32 = std::is_same<T, float>::value;
   using LY = GemmLayout<TN, NB>;
   constexpr int BK = kRowBytes / static_cast<int>(sizeof(T));   // K elements per stage

@@ -69,6 +69,7 @@ template <int TNH, int EPI, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                              const __grid_constant__ CUtensorMap tmB1, const GemmArgs args) {
+  pdl_enter();
   using T = __nv_bfloat16;
   using LY = PairLayout<TNH>;
   constexpr int BK = kRowBytes / 2;

@@ -104,6 +104,7 @@ struct MxScaleJob {
 };
 
 __global__ void __launch_bounds__(256) mx_scale_relayout_kernel(MxScaleJob job) {
+  pdl_enter();
   const int m = blockIdx.y;
   const int N = job.rows[m], K = job.kdim[m];
   const int KS = K / 32, KB = (K + 63) / 64;
@@ -132,6 +133,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
     grouped_gemm_pair_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP0,
                                 const __grid_constant__ CUtensorMap tmP1, const __grid_constant__ CUtensorMap tmS0,
                                 const __grid_constant__ CUtensorMap tmS1, const GemmArgs args) {
+  pdl_enter();
   using T = __nv_bfloat16;
   using LY = PairMxLayout<TNH>;
   constexpr int BK = kRowBytes / 2;        // 64 K elements per step

@@ -171,6 +171,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
                                 const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmX16,
                                 const GemmArgs args) {
+  pdl_enter();
   using LY = WmLayout;
   constexpr int BK = kRowBytes / 2;
   constexpr int KSTEPS = kRowBytes / 32;

@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(256) router_topk_partials_kernel(const float* 
                                                                    const T* __restrict__ br, int Tn, int E, int k,
                                                                    int32_t* __restrict__ ids,
                                                                    float* __restrict__ wout) {
+  pdl_enter();
   constexpr int TPB = 256 / P;                       // tokens per block
   __shared__ float bias[256];
   __shared__ float lv[P][8][TPB];
@@ -238,6 +239,7 @@ template <typename T>
 __global__ void __launch_bounds__(kRouterWarps * 32)
     router_simt_kernel(const T* __restrict__ x, const T* __restrict__ wr, const T* __restrict__ br, int D, int E,
                        int k, int32_t* __restrict__ ids, float* __restrict__ wout) {
+  pdl_enter();
   __shared__ float logits[256];
   __shared__ uint4 xs[kRouterMaxChunks];
   const int t = blockIdx.x;
@@ -283,16 +285,16 @@ cudaError_t router_topk(const Launch& L, bool bf16, int64_t T, int D, int E, int
     const __nv_bfloat16* br = static_cast<const __nv_bfloat16*>(b_router);
     const int Ti = static_cast<int>(T);
     if (E <= 32)
-      router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 1><<<(Ti + 255) / 256, 256, 0, L.stream>>>(
+      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 1>, dim3((Ti + 255) / 256), dim3(256), 0, L.stream, 
           partial, br, Ti, E, k, ids, w);
     else if (E <= 64)
-      router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 2><<<(Ti + 127) / 128, 256, 0, L.stream>>>(
+      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 2>, dim3((Ti + 127) / 128), dim3(256), 0, L.stream, 
           partial, br, Ti, E, k, ids, w);
     else if (E <= 128)
-      router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 4><<<(Ti + 63) / 64, 256, 0, L.stream>>>(
+      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 4>, dim3((Ti + 63) / 64), dim3(256), 0, L.stream, 
           partial, br, Ti, E, k, ids, w);
     else
-      router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 8><<<(Ti + 31) / 32, 256, 0, L.stream>>>(
+      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 8>, dim3((Ti + 31) / 32), dim3(256), 0, L.stream, 
           partial, br, Ti, E, k, ids, w);
     count_launch();
     return cudaGetLastError();
@@ -300,11 +302,11 @@ cudaError_t router_topk(const Launch& L, bool bf16, int64_t T, int D, int E, int
   if (bf16 && T >= 256) return router_tc(L, T, D, E, k, x, w_router, b_router, ids, w);
   const dim3 grid(static_cast<unsigned>(T));
   if (bf16)
-    router_simt_kernel<__nv_bfloat16><<<grid, kRouterWarps * 32, 0, L.stream>>>(
+    pdl_launch(router_simt_kernel<__nv_bfloat16>, dim3(grid), dim3(kRouterWarps * 32), 0, L.stream, 
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
         static_cast<const __nv_bfloat16*>(b_router), D, E, k, ids, w);
   else
-    router_simt_kernel<float><<<grid, kRouterWarps * 32, 0, L.stream>>>(
+    pdl_launch(router_simt_kernel<float>, dim3(grid), dim3(kRouterWarps * 32), 0, L.stream, 
         static_cast<const float*>(x), static_cast<const float*>(w_router), static_cast<const float*>(b_router), D,
         E, k, ids, w);
   count_launch();
@@ -349,6 +351,7 @@ __device__ __forceinline__ void build_masks(uint32_t (*mask)[256], const int32_t
 
 __global__ void __launch_bounds__(kChunk) permute_count_kernel(const int32_t* __restrict__ ids, int T, int k, int E,
                                                                int nchunks, int32_t* __restrict__ chunk_cnt) {
+  pdl_enter();
   __shared__ uint32_t mask[kChunkWarps][256];
   build_masks(mask, ids, T, k, E);
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -362,6 +365,7 @@ __global__ void __launch_bounds__(kChunk) permute_count_kernel(const int32_t* __
 // Exclusive scan over the expert-major (expert, chunk) counts; one block.
 __global__ void __launch_bounds__(1024) permute_scan_kernel(const int32_t* __restrict__ cnt, int n, int E, int nchunks,
                                                             int32_t* __restrict__ base, int32_t* __restrict__ expert_off) {
+  pdl_enter();
   __shared__ int warp_tot[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (n + blockDim.x - 1) / blockDim.x;
@@ -401,6 +405,7 @@ __global__ void __launch_bounds__(kChunk) permute_scatter_kernel(const int32_t* 
                                                                  int nchunks, const int32_t* __restrict__ base,
                                                                  int32_t* __restrict__ row_of_slot,
                                                                  int32_t* __restrict__ slot_of_row) {
+  pdl_enter();
   __shared__ uint32_t mask[kChunkWarps][256];
   build_masks(mask, ids, T, k, E);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -425,6 +430,7 @@ __global__ void __launch_bounds__(kChunk) permute_scatter_kernel(const int32_t* 
 // x_perm[r] = x[slot_of_row[r] / k], one warp per row, 16-byte vectors.
 __global__ void permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ slot_of_row, int R,
                                       int k, int T, int vec_per_row, uint4* __restrict__ x_perm) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -451,6 +457,7 @@ __global__ void __launch_bounds__(kChunk) permute_small_kernel(const int32_t* __
                                                                int32_t* __restrict__ row_of_slot,
                                                                int32_t* __restrict__ slot_of_row,
                                                                uint4* __restrict__ x_perm) {
+  pdl_enter();
   __shared__ uint32_t mask[kChunkWarps][256];
   __shared__ int base[257];
   __shared__ int sor[kSmallMaxRows];
@@ -541,7 +548,7 @@ cudaError_t permute(const Launch& L, bool bf16, int64_t T, int D, int E, int k, 
     // one CTA builds the maps; it also copies the rows when there are few of them
     const bool rows = x != nullptr && x_perm != nullptr;
     const bool copy_here = rows && T * k <= kSmallCopyRows;
-    permute_small_kernel<<<1, kChunk, 0, L.stream>>>(ids, static_cast<int>(T), k, E,
+    pdl_launch(permute_small_kernel, dim3(1), dim3(kChunk), 0, L.stream, ids, static_cast<int>(T), k, E,
                                                      copy_here ? static_cast<const uint4*>(x) : nullptr,
                                                      D * (bf16 ? 2 : 4) / 16, expert_off, row_of_slot, slot_of_row,
                                                      copy_here ? static_cast<uint4*>(x_perm) : nullptr);
@@ -550,9 +557,9 @@ cudaError_t permute(const Launch& L, bool bf16, int64_t T, int D, int E, int k, 
   } else {
     int32_t* cnt = scratch;
     int32_t* base = scratch + static_cast<size_t>(nchunks) * E;
-    permute_count_kernel<<<nchunks, kChunk, 0, L.stream>>>(ids, static_cast<int>(T), k, E, nchunks, cnt);
-    permute_scan_kernel<<<1, 1024, 0, L.stream>>>(cnt, nchunks * E, E, nchunks, base, expert_off);
-    permute_scatter_kernel<<<nchunks, kChunk, 0, L.stream>>>(ids, static_cast<int>(T), k, E, nchunks, base,
+    pdl_launch(permute_count_kernel, dim3(nchunks), dim3(kChunk), 0, L.stream, ids, static_cast<int>(T), k, E, nchunks, cnt);
+    pdl_launch(permute_scan_kernel, dim3(1), dim3(1024), 0, L.stream, cnt, nchunks * E, E, nchunks, base, expert_off);
+    pdl_launch(permute_scatter_kernel, dim3(nchunks), dim3(kChunk), 0, L.stream, ids, static_cast<int>(T), k, E, nchunks, base,
                                                              row_of_slot, slot_of_row);
     count_launch(3);
   }
@@ -561,7 +568,7 @@ cudaError_t permute(const Launch& L, bool bf16, int64_t T, int D, int E, int k, 
     const int vpr = D * (bf16 ? 2 : 4) / 16;
     const int warps_needed = R;
     const int blocks = static_cast<int>(std::min<int64_t>((warps_needed + 7) / 8, int64_t(L.num_sms) * 8));
-    permute_gather_kernel<<<blocks, 256, 0, L.stream>>>(static_cast<const uint4*>(x), slot_of_row, R, k,
+    pdl_launch(permute_gather_kernel, dim3(blocks), dim3(256), 0, L.stream, static_cast<const uint4*>(x), slot_of_row, R, k,
                                                        static_cast<int>(T), vpr, static_cast<uint4*>(x_perm));
     count_launch();
   }
@@ -574,6 +581,7 @@ cudaError_t permute(const Launch& L, bool bf16, int64_t T, int D, int E, int k, 
 template <typename T>
 __global__ void combine_gather_kernel(const T* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
                                       const float* __restrict__ w, int Tn, int k, int D, T* __restrict__ y) {
+  pdl_enter();
   const int nv = D / 8;
   const int64_t total = static_cast<int64_t>(Tn) * nv;
   const int R = Tn * k;
@@ -600,6 +608,7 @@ __global__ void combine_gather_kernel(const T* __restrict__ y_perm, const int32_
 
 template <typename T>
 __global__ void combine_slots_kernel(const float* __restrict__ ys, int Tn, int k, int D, T* __restrict__ y) {
+  pdl_enter();
   const int nv = D / 8;
   const int64_t total = static_cast<int64_t>(Tn) * nv;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
@@ -627,11 +636,11 @@ cudaError_t combine_gather(const Launch& L, bool bf16, int64_t T, int D, int k, 
   if (T == 0) return cudaSuccess;
   const int blocks = elementwise_blocks(L, T * (D / 8));
   if (bf16)
-    combine_gather_kernel<__nv_bfloat16><<<blocks, 256, 0, L.stream>>>(
+    pdl_launch(combine_gather_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, L.stream, 
         static_cast<const __nv_bfloat16*>(y_perm), row_of_slot, w, static_cast<int>(T), k, D,
         static_cast<__nv_bfloat16*>(y));
   else
-    combine_gather_kernel<float><<<blocks, 256, 0, L.stream>>>(static_cast<const float*>(y_perm), row_of_slot, w,
+    pdl_launch(combine_gather_kernel<float>, dim3(blocks), dim3(256), 0, L.stream, static_cast<const float*>(y_perm), row_of_slot, w,
                                                               static_cast<int>(T), k, D, static_cast<float*>(y));
   count_launch();
   return cudaGetLastError();
@@ -641,10 +650,10 @@ cudaError_t combine_slots(const Launch& L, bool bf16, int64_t T, int D, int k, c
   if (T == 0) return cudaSuccess;
   const int blocks = elementwise_blocks(L, T * (D / 8));
   if (bf16)
-    combine_slots_kernel<__nv_bfloat16><<<blocks, 256, 0, L.stream>>>(
+    pdl_launch(combine_slots_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, L.stream, 
         static_cast<const float*>(ys), static_cast<int>(T), k, D, static_cast<__nv_bfloat16*>(y));
   else
-    combine_slots_kernel<float><<<blocks, 256, 0, L.stream>>>(static_cast<const float*>(ys), static_cast<int>(T),
+    pdl_launch(combine_slots_kernel<float>, dim3(blocks), dim3(256), 0, L.stream, static_cast<const float*>(ys), static_cast<int>(T),
                                                              k, D, static_cast<float*>(y));
   count_launch();
   return cudaGetLastError();

@@ -18,6 +18,7 @@ template <int EPI>
 __global__ void __launch_bounds__(256)
     simt_grouped_gemm_f32(const float* __restrict__ A, const float* __restrict__ B0, const float* __restrict__ B1,
                           const GemmArgs args) {
+  pdl_enter();
   constexpr bool kTwo = EPI == EPI_SWIGLU;
   __shared__ float sa[kSimtBK][kSimtBM + 4];
   __shared__ float sb0[kSimtBK][kSimtBN + 4];
