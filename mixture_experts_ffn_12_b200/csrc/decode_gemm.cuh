@@ -21,20 +21,22 @@
 
 namespace moe {
 
+constexpr int kDecKBS = 1;           // 64-wide K blocks per stage
 constexpr int kDecStages = 10;       // one CTA per SM
 constexpr int kDecStagesDual = 5;    // two CTAs per SM
 constexpr int kDecTmemCols = 64;   // two accumulators of NTOK = 32 columns
 
-template <int NTOK>
+// A stage holds KBS consecutive 64-wide K blocks: [KBS weight tiles][KBS token tiles].
+template <int NTOK, int KBS = 1>
 struct DecLayout {
-  static constexpr int W_BYTES = 128 * kRowBytes;     // 16 KB of weight rows per K step
+  static constexpr int W_BYTES = 128 * kRowBytes;     // 16 KB of weight rows per K block
   static constexpr int X_BYTES = NTOK * kRowBytes;
-  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+  static constexpr int STAGE_BYTES = KBS * (W_BYTES + X_BYTES);
   static constexpr int UP_BYTES = 64 * NTOK * 4;      // up values handed to the gate warps
   static constexpr int EXTRA = 1024 + 2560;   // alignment slack; barriers, unit and group offsets (2.3 KB)
   static constexpr int smem_bytes(int stages) { return stages * STAGE_BYTES + UP_BYTES + EXTRA; }
   static_assert(NTOK % 16 == 0 && NTOK <= 256, "MMA N");
-  static_assert(2 * (STAGE_BYTES * kDecStagesDual + UP_BYTES + EXTRA + 1024) <= 233472,
+  static_assert(KBS > 1 || 2 * (STAGE_BYTES * kDecStagesDual + UP_BYTES + EXTRA + 1024) <= 233472,
                 "two CTAs per SM (plus 1 KB reserved each) fit the 228 KB of shared memory");
 };
 
@@ -64,13 +66,13 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const int* unit_off, cons
 }
 
 // EPI_SWIGLU: tmW0 = W_gate, tmW1 = W_up (boxes of 64 rows); EPI_BIAS / EPI_BIAS_WSCATTER: tmW0 = W_down (128 rows).
-template <int EPI, int NTOK, int STAGES>
+template <int EPI, int NTOK, int STAGES, int KBS = 1>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
                        const __grid_constant__ CUtensorMap tmX, const GemmArgs args) {
   pdl_enter();
   using T = __nv_bfloat16;
-  using LY = DecLayout<NTOK>;
+  using LY = DecLayout<NTOK, KBS>;
   constexpr int BK = kRowBytes / 2;
   constexpr int KSTEPS = kRowBytes / 32;
   constexpr bool kGateUp = EPI == EPI_SWIGLU;
@@ -97,6 +99,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int G = args.num_groups;
   const int FB = (args.n_out + FBW - 1) / FBW;
   const int KB = (args.k_dim + BK - 1) / BK;
+  const int KSTEP_STAGES = (KB + KBS - 1) / KBS;      // stages per unit (blocks past K read zeros)
   const uint64_t lim = args.wait_limit_ns;
 
   if (threadIdx.x == 0) {
@@ -170,18 +173,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
         const UnitInfo ui = unit(u);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int ks = 0; ks < KSTEP_STAGES; ++ks) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], tx_bytes);
-          uint8_t* sw = smem + s * LY::STAGE_BYTES;
-          uint8_t* sx = sw + LY::W_BYTES;
-          if (kGateUp) {
-            tma_load_3d(sw, &tmW0, &full[s], kb * BK, ui.f0, ui.g);
-            tma_load_3d(sw + 64 * kRowBytes, &tmW1, &full[s], kb * BK, ui.f0, ui.g);
-          } else {
-            tma_load_3d(sw, &tmW0, &full[s], kb * BK, ui.f0, ui.g);
+#pragma unroll
+          for (int b = 0; b < KBS; ++b) {
+            const int kb = ks * KBS + b;
+            uint8_t* sw = smem + s * LY::STAGE_BYTES + b * LY::W_BYTES;
+            uint8_t* sx = smem + s * LY::STAGE_BYTES + KBS * LY::W_BYTES + b * LY::X_BYTES;
+            if (kGateUp) {
+              tma_load_3d(sw, &tmW0, &full[s], kb * BK, ui.f0, ui.g);
+              tma_load_3d(sw + 64 * kRowBytes, &tmW1, &full[s], kb * BK, ui.f0, ui.g);
+            } else {
+              tma_load_3d(sw, &tmW0, &full[s], kb * BK, ui.f0, ui.g);
+            }
+            tma_load_2d(sx, &tmX, &full[s], kb * BK, ui.m0);
           }
-          tma_load_2d(sx, &tmX, &full[s], kb * BK, ui.m0);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -209,15 +216,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, lim)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * NTOK);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int ks = 0; ks < KSTEP_STAGES; ++ks) {
           if (!mbar_wait(&full[s], ph, abort_flag, lim)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t w_addr = smem_u32(smem + s * LY::STAGE_BYTES);
-          const uint32_t x_addr = w_addr + LY::W_BYTES;
+          const uint32_t stage_addr = smem_u32(smem + s * LY::STAGE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < KSTEPS; ++kk)
-            tc_mma<false>(d_tmem, sw128_kmajor_desc(w_addr + kk * 32), sw128_kmajor_desc(x_addr + kk * 32), idesc,
-                          (kb | kk) != 0 ? 1u : 0u);
+          for (int b = 0; b < KBS; ++b) {
+            const uint32_t w_addr = stage_addr + b * LY::W_BYTES;
+            const uint32_t x_addr = stage_addr + KBS * LY::W_BYTES + b * LY::X_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk)
+              tc_mma<false>(d_tmem, sw128_kmajor_desc(w_addr + kk * 32), sw128_kmajor_desc(x_addr + kk * 32), idesc,
+                            (ks | b | kk) != 0 ? 1u : 0u);
+          }
           tc_commit(&empty[s]);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
         }

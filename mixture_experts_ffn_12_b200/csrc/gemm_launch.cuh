@@ -211,8 +211,8 @@ constexpr int kDecTok = 32;
 template <int EPI, int STAGES>
 static cudaError_t launch_decode_st(const Launch& L, const CUtensorMap& w0, const CUtensorMap& w1,
                                     const CUtensorMap& x, const GemmArgs& args, int grid) {
-  auto kern = decode_gemm_kernel<EPI, kDecTok, STAGES>;
-  constexpr int smem = DecLayout<kDecTok>::smem_bytes(STAGES);
+  auto kern = decode_gemm_kernel<EPI, kDecTok, STAGES, kDecKBS>;
+  constexpr int smem = DecLayout<kDecTok, kDecKBS>::smem_bytes(STAGES);
   static_assert(smem <= 232448, "shared memory budget");
   int dev = 0;
   cudaGetDevice(&dev);

@@ -377,8 +377,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
     const int grp = cw / kMxGroupWarps;
     const int ct = (cw % kMxGroupWarps) * 32 + lane;     // 0..127 within the group
     const uint32_t conv_leader = mapa_shared(smem_u32(conv), 0);
-    const int c = ct & 7;                                // 4-byte chunk of a 32-byte packed row (8 codes)
-    const int r0 = ct >> 3;                              // rows r0, r0 + 16, ...
     // this cluster's K steps, numbered across its tiles like the producers walk them
     const int my_tiles = cluster < total ? (total - cluster + nclusters - 1) / nclusters : 0;
     const int steps = my_tiles * KB;
@@ -392,13 +390,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
       const uint8_t* sp = pring + p * LY::SLOT_BYTES;
       const uint8_t* ss = sp + LY::P_BYTES;
       uint8_t* sb = smem + s * LY::STAGE_BYTES + LY::A_BYTES;
+      // a task is half a packed row: 16 bytes = 32 codes = one scale block, i.e.
+      // four 16-byte chunks (8 bf16 each) of the swizzled bf16 row
 #pragma unroll
-      for (int q = 0; q < (TNH + 15) / 16; ++q) {
-        const int r = r0 + 16 * q;
-        if (r < TNH) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(sp + r * 32 + c * 4);
-          const uint4 v = mxfp4_decode8(w, e8m0_to_bf16x2(ss[r * 2 + (c >> 2)]));
-          *reinterpret_cast<uint4*>(sb + r * kRowBytes + ((c ^ (r & 7)) << 4)) = v;
+      for (int q = 0; q < (2 * TNH + 127) / 128; ++q) {
+        const int tk = ct + 128 * q;
+        if (tk < 2 * TNH) {
+          const int r = tk >> 1, h = tk & 1, x = r & 7;
+          const uint4 w4 = *reinterpret_cast<const uint4*>(sp + r * 32 + h * 16);
+          const __nv_bfloat162 sc = e8m0_to_bf16x2(ss[r * 2 + h]);
+          uint8_t* row = sb + r * kRowBytes;
+          *reinterpret_cast<uint4*>(row + (((4 * h + 0) ^ x) << 4)) = mxfp4_decode8(w4.x, sc);
+          *reinterpret_cast<uint4*>(row + (((4 * h + 1) ^ x) << 4)) = mxfp4_decode8(w4.y, sc);
+          *reinterpret_cast<uint4*>(row + (((4 * h + 2) ^ x) << 4)) = mxfp4_decode8(w4.z, sc);
+          *reinterpret_cast<uint4*>(row + (((4 * h + 3) ^ x) << 4)) = mxfp4_decode8(w4.w, sc);
         }
       }
       fence_proxy_async_smem();     // generic-proxy stores -> visible to the tensor core

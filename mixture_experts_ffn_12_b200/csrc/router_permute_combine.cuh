@@ -31,6 +31,7 @@ namespace moe {
 constexpr int kRouterWarps = 32;   // one block per token: a warp per expert for E <= 32
 constexpr int kRouterSplits = 4;   // K ranges of the tensor-core router inside the fused layer
 constexpr int kRouterMaxChunks = 1024;   // x row staged in shared memory: D * elem <= 16 KB
+constexpr int kTopkExpertsPerThread = 8; // router top-k after the K split: experts scanned per thread
 
 // Dot product of a row of x (staged in shared memory, or in global memory) with a weight row in global
 // memory; lanes stride over 16-byte chunks.  The weight loads of a batch are all
@@ -129,7 +130,7 @@ __device__ __forceinline__ void warp_topk_softmax(float (&v)[8], int lane, int E
 
 // Fused-layer router tail: sum of the K-range partial logits (partial[split][e][t])
 // + router bias, top-k and the softmax over the k selected.  P threads per token
-// (P = power of two >= E / 32), each scanning up to 32 experts: thread (part, t)
+// (P = power of two >= E / 8), each scanning up to 8 experts: thread (part, t)
 // with t fastest in the block, so each expert's loads are coalesced across tokens.
 // Each thread keeps a running top-k of its experts in index order (strict '>'
 // keeps the lower index first on ties); part 0 merges the P lists through shared
@@ -154,7 +155,7 @@ __global__ void __launch_bounds__(256) router_topk_partials_kernel(const float* 
 #pragma unroll
   for (int j = 0; j < 8; ++j) { tv[j] = -INFINITY; tix[j] = 0x7fffffff; }
   const size_t plane = static_cast<size_t>(E) * Tn;
-  const int e_begin = part * 32, e_end = min(E, e_begin + 32);
+  const int e_begin = part * kTopkExpertsPerThread, e_end = min(E, e_begin + kTopkExpertsPerThread);
   if (tv_ok) {
 #pragma unroll 1
     for (int e0 = e_begin; e0 < e_end; e0 += 8) {
@@ -284,18 +285,25 @@ cudaError_t router_topk(const Launch& L, bool bf16, int64_t T, int D, int E, int
     if (e != cudaSuccess) return e;
     const __nv_bfloat16* br = static_cast<const __nv_bfloat16*>(b_router);
     const int Ti = static_cast<int>(T);
-    if (E <= 32)
-      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 1>, dim3((Ti + 255) / 256), dim3(256), 0, L.stream, 
-          partial, br, Ti, E, k, ids, w);
-    else if (E <= 64)
-      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 2>, dim3((Ti + 127) / 128), dim3(256), 0, L.stream, 
-          partial, br, Ti, E, k, ids, w);
-    else if (E <= 128)
-      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 4>, dim3((Ti + 63) / 64), dim3(256), 0, L.stream, 
-          partial, br, Ti, E, k, ids, w);
+    const int parts = (E + kTopkExpertsPerThread - 1) / kTopkExpertsPerThread;
+    if (parts <= 1)
+      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 1>, dim3((Ti + 255) / 256), dim3(256), 0,
+                 L.stream, partial, br, Ti, E, k, ids, w);
+    else if (parts <= 2)
+      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 2>, dim3((Ti + 127) / 128), dim3(256), 0,
+                 L.stream, partial, br, Ti, E, k, ids, w);
+    else if (parts <= 4)
+      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 4>, dim3((Ti + 63) / 64), dim3(256), 0,
+                 L.stream, partial, br, Ti, E, k, ids, w);
+    else if (parts <= 8)
+      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 8>, dim3((Ti + 31) / 32), dim3(256), 0,
+                 L.stream, partial, br, Ti, E, k, ids, w);
+    else if (parts <= 16)
+      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 16>, dim3((Ti + 15) / 16), dim3(256), 0,
+                 L.stream, partial, br, Ti, E, k, ids, w);
     else
-      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 8>, dim3((Ti + 31) / 32), dim3(256), 0, L.stream, 
-          partial, br, Ti, E, k, ids, w);
+      pdl_launch(router_topk_partials_kernel<__nv_bfloat16, kRouterSplits, 32>, dim3((Ti + 7) / 8), dim3(256), 0,
+                 L.stream, partial, br, Ti, E, k, ids, w);
     count_launch();
     return cudaGetLastError();
   }
@@ -443,7 +451,21 @@ __global__ void permute_gather_kernel(const uint4* __restrict__ x, const int32_t
     }
     const uint4* src = x + static_cast<size_t>(t) * vec_per_row;
     uint4* dst = x_perm + static_cast<size_t>(r) * vec_per_row;
-    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+    // batches of kGatherBatch independent loads per lane before the stores
+    constexpr int kGatherBatch = 12;
+    for (int v0 = lane; v0 < vec_per_row; v0 += 32 * kGatherBatch) {
+      uint4 buf[kGatherBatch];
+#pragma unroll
+      for (int u = 0; u < kGatherBatch; ++u) {
+        const int v = v0 + 32 * u;
+        if (v < vec_per_row) buf[u] = src[v];
+      }
+#pragma unroll
+      for (int u = 0; u < kGatherBatch; ++u) {
+        const int v = v0 + 32 * u;
+        if (v < vec_per_row) dst[v] = buf[u];
+      }
+    }
   }
 }
 
@@ -615,13 +637,18 @@ __global__ void combine_slots_kernel(const float* __restrict__ ys, int Tn, int k
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int t = static_cast<int>(i / nv);
     const int c = static_cast<int>(i - static_cast<int64_t>(t) * nv) * 8;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j = 0; j < k; ++j) {
-      float v[8];
-      load8<float>(ys + (static_cast<size_t>(t) * k + j) * D + c, v);
+    // all k rows' loads first, then the sum in slot order
+    float v[8][8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] += v[q];
-    }
+    for (int j = 0; j < 8; ++j)
+      if (j < k) load8<float>(ys + (static_cast<size_t>(t) * k + j) * D + c, v[j]);
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < k) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] += v[j][q];
+      }
     store8<T>(y + static_cast<size_t>(t) * D + c, acc);
   }
 }
