@@ -40,6 +40,11 @@ PAIR_RAGGED = W.tiny_spec(T=900, D=256, E=5, k=2, F=272, dtype="bf16", cfg_id=20
                           router_w_std=0.2)
 
 SMALL_SPECS = [W.TINY_FP32, RAGGED_BF16, RAGGED_F32, WIDE_K, ONE_EXPERT, MXFP4_SMALL, PAIR_RAGGED]
+
+# many experts: the K-split router with 16 / 32 threads per token in its top-k (E = 128 / 256),
+# 256 expert groups in the GEMMs (the maximum), k = 8 (the maximum)
+MANY_EXPERTS = [W.tiny_spec(T=300, D=512, E=128, k=8, F=96, dtype="bf16", cfg_id=207, router_w_std=0.2),
+                W.tiny_spec(T=520, D=1024, E=256, k=8, F=64, dtype="bf16", cfg_id=208, router_w_std=0.2)]
 DECODE_SPECS = [W.gptoss20b_decode(t) for t in W.GPTOSS20B_DECODE_T]
 
 
@@ -227,6 +232,32 @@ def test_layer_forward_all_tokens(api, spec):
     check_output(f64(y), ref["y"], tol_for(spec), spec.dtype == "bf16")
 
 
+@pytest.mark.parametrize("spec", MANY_EXPERTS, ids=lambda s: s.name)
+def test_layer_forward_many_experts(api, spec):
+    layer = layer_for(spec)
+    y, gid, _ = _run_layer(api, spec, layer)
+    ref = O.layer_tokens(layer, np.arange(spec.T), spec.k, spec.limit, spec.alpha)
+    check_ids(gid, ref["ids"], ref["logits"])
+    check_output(f64(y), ref["y"], tol_for(spec), True)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_layer_forward_zero_tokens(api, dtype):
+    """T = 0: MOE_OK, nothing launched, nothing written."""
+    from mixture_experts_ffn_12_b200 import _lib
+    spec = W.tiny_spec(T=0, D=64, E=4, k=2, F=32, dtype=dtype, cfg_id=209)
+    layer = layer_for(spec)
+    d = dev(layer, api)
+    lib = _lib.load()
+    before = lib.moe_launch_count()
+    y = api.layer_forward(api.config_from_spec(spec), d["x"], d["w_router"], d["b_router"],
+                          api.expert_weights_from(d))
+    torch.cuda.synchronize()
+    assert tuple(y.shape) == (0, spec.D)
+    assert lib.moe_launch_count() == before
+    assert api.last_device_error() == 0
+
+
 @pytest.mark.parametrize("spec", [W.GPTOSS20B_PREFILL, W.GPTOSS20B_MXFP4, W.GPTOSS120B_SKEWED],
                          ids=lambda s: s.name)
 def test_layer_forward_full_size_sampled(api, spec):
@@ -307,6 +338,23 @@ def test_cuda_graph_replay_matches_eager(api):
     torch.cuda.synchronize()
     assert api.last_device_error() == 0
     assert torch.equal(y_graph, y_eager)
+
+
+def test_run_host_batches_matches_layer_calls(api):
+    """The pipelined host->device->host runner gives each batch the layer's own output."""
+    spec = RAGGED_BF16
+    layer = layer_for(spec)
+    d = dev(layer, api)
+    moe = api.MoELayer(api.config_from_spec(spec), d["w_router"], d["b_router"], api.expert_weights_from(d))
+    xs = [torch.roll(d["x"], shifts=7 * i, dims=0).contiguous() for i in range(5)]
+    want = [moe(x).cpu() for x in xs]
+    xs_host = [x.cpu().pin_memory() for x in xs]
+    ys_host = [torch.empty_like(w).pin_memory() for w in want]
+    moe.run_host_batches(xs_host, ys_host)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    for got, w in zip(ys_host, want):
+        assert torch.equal(got, w)
 
 
 def test_mxfp4_matches_bf16_path_on_dequantised_weights(api):
