@@ -278,24 +278,20 @@ def run_ours(args, rank, world, local_rank):
     stage_ms = {name: statistics.mean(ev[i][s].elapsed_time(ev[i][n + s]) for i in range(K))
                 for s, name in enumerate(STAGES)}
 
-    # end to end: pinned host input -> device, layer, device -> pinned host output, every step
-    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
-    x_host.copy_(x)
-    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-    x_dev = torch.empty_like(x)
-    for _ in range(3):
-        x_dev.copy_(x_host, non_blocking=True)
-        moe(x_dev, y=y)
-        y_host.copy_(y, non_blocking=True)
+    # end to end through MoELayer.run_host_batches: every step copies its input from
+    # pinned host memory and its output back to pinned host memory; the copies of
+    # neighbouring steps overlap the forward (three streams, double-buffered)
+    Ke = max(5, K // 4)
+    xs_host = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for _ in range(2)]
+    for xh in xs_host:
+        xh.copy_(x)
+    ys_host = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for _ in range(2)]
+    moe.run_host_batches([xs_host[i % 2] for i in range(3)], [ys_host[i % 2] for i in range(3)])
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    Ke = max(5, K // 4)
     e0.record(stream)
-    for _ in range(Ke):
-        x_dev.copy_(x_host, non_blocking=True)
-        moe(x_dev, y=y)
-        y_host.copy_(y, non_blocking=True)
+    moe.run_host_batches([xs_host[i % 2] for i in range(Ke)], [ys_host[i % 2] for i in range(Ke)])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()

@@ -226,3 +226,52 @@ class MoELayer:
             layer_forward(self.cfg, x, self.w_router, self.b_router, self.experts, y=y, ws=ws,
                           topk_ids=topk_ids, topk_w=topk_w)
         return g.replay, y
+
+    def run_host_batches(self, xs_host, ys_host) -> None:
+        """Run the layer on a sequence of pinned host batches, results into pinned host buffers.
+
+        Batch i's host->device copy, forward and device->host copy go on three
+        streams with two device buffers each way, so the copies of neighbouring
+        batches overlap this batch's forward (PCIe is full duplex).  Ordering:
+        copy-in(i) after forward(i-2) released its input buffer; forward(i) after
+        copy-in(i) and after copy-out(i-2) released its output buffer; copy-out(i)
+        after forward(i).  Returns when everything has been queued; the caller
+        synchronises.  All batches must have the same shape.
+        """
+        if len(xs_host) == 0:
+            return
+        dev = self.w_router.device
+        T, D = xs_host[0].shape
+        xd = [torch.empty((T, D), dtype=xs_host[0].dtype, device=dev) for _ in range(2)]
+        yd = [torch.empty((T, self.cfg.hidden_size), dtype=xs_host[0].dtype, device=dev) for _ in range(2)]
+        s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        cur = torch.cuda.current_stream(dev)
+        for st in (s_in, s_run, s_out):
+            st.wait_stream(cur)
+        copied = [torch.cuda.Event() for _ in range(2)]
+        ran = [torch.cuda.Event() for _ in range(2)]
+        drained = [torch.cuda.Event() for _ in range(2)]
+        self.workspace(T)
+        for i, (xh, yh) in enumerate(zip(xs_host, ys_host)):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ran[b])
+                xd[b].copy_(xh, non_blocking=True)
+                copied[b].record(s_in)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(copied[b])
+                if i >= 2:
+                    s_run.wait_event(drained[b])
+                self(xd[b], y=yd[b])
+                ran[b].record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ran[b])
+                yh.copy_(yd[b], non_blocking=True)
+                drained[b].record(s_out)
+        for st in (s_in, s_run, s_out):
+            cur.wait_stream(st)
+        for t in xd + yd:
+            t.record_stream(s_in)
+            t.record_stream(s_run)
+            t.record_stream(s_out)
