@@ -245,37 +245,44 @@ def run_ours(args, rank, world, local_rank):
     if api.last_device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
 
-    # per-step stage events, recorded by the library on this stream
+    # timed steps: back-to-back layer calls, nothing else on the stream
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(STAGES))] for _ in range(K)]
-    for row in ev:
-        for e in row:
-            e.record(stream)   # materialise the handles
-    torch.cuda.synchronize()
-    handles = [[ctypes_ptr(e.cuda_event) for e in row] for row in ev]
-    n = len(STAGES)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
     sampler = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
     with sampler:
         launches0 = lib.moe_launch_count()
         t0.record(stream)
-        for i in range(K):
-            starts = (_lib.ctypes.c_void_p * n)(*handles[i][:n])
-            stops = (_lib.ctypes.c_void_p * n)(*handles[i][n:])
-            lib.moe_set_stage_events(starts, stops, n)
+        for _ in range(K):
             moe(x, y=y)
         t1.record(stream)
-        lib.moe_set_stage_events(None, None, 0)
         launches = lib.moe_launch_count() - launches0
         torch.cuda.synchronize()
     barrier()
     ms_total = max_over_ranks(t0.elapsed_time(t1))
     if api.last_device_error() != 0:
         raise RuntimeError("device error word set during the timed steps")
-    stage_ms = {name: statistics.mean(ev[i][s].elapsed_time(ev[i][n + s]) for i in range(K))
+
+    # stage times (and the gate/up kernel's time for the roofline) from a separate pass:
+    # the library records CUDA events on this stream around each stage, which adds
+    # event records between the kernels, so this pass is not the one `value` comes from
+    Ks = min(K, 50)
+    n = len(STAGES)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(Ks)]
+    for row in ev:
+        for e in row:
+            e.record(stream)   # materialise the handles
+    torch.cuda.synchronize()
+    handles = [[ctypes_ptr(e.cuda_event) for e in row] for row in ev]
+    for i in range(Ks):
+        starts = (_lib.ctypes.c_void_p * n)(*handles[i][:n])
+        stops = (_lib.ctypes.c_void_p * n)(*handles[i][n:])
+        lib.moe_set_stage_events(starts, stops, n)
+        moe(x, y=y)
+    lib.moe_set_stage_events(None, None, 0)
+    torch.cuda.synchronize()
+    stage_ms = {name: statistics.mean(ev[i][s].elapsed_time(ev[i][n + s]) for i in range(Ks))
                 for s, name in enumerate(STAGES)}
 
     # end to end through MoELayer.run_host_batches: every step copies its input from
