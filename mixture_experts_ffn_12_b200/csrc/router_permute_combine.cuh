@@ -637,18 +637,13 @@ __global__ void combine_slots_kernel(const float* __restrict__ ys, int Tn, int k
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int t = static_cast<int>(i / nv);
     const int c = static_cast<int>(i - static_cast<int64_t>(t) * nv) * 8;
-    // all k rows' loads first, then the sum in slot order
-    float v[8][8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j < k) load8<float>(ys + (static_cast<size_t>(t) * k + j) * D + c, v[j]);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < k; ++j) {
+      float v[8];
+      load8<float>(ys + (static_cast<size_t>(t) * k + j) * D + c, v);
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j < k) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] += v[j][q];
-      }
+      for (int q = 0; q < 8; ++q) acc[q] += v[q];
+    }
     store8<T>(y + static_cast<size_t>(t) * D + c, acc);
   }
 }
