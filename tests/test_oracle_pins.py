@@ -284,6 +284,30 @@ def test_unrouted_expert_contributes_nothing():
     np.testing.assert_array_equal(ref2["y"], ref["y"])
 
 
+def test_identical_experts_give_the_dense_mlp():
+    """If every expert has the same weights and biases, routing cannot matter: the softmax
+    weights sum to 1, so every token's output is that one dense MLP's output (a scalar
+    triple loop), whatever the router picks."""
+    spec = W.tiny_spec(T=11, D=16, E=5, k=3, F=24, dtype="f32", expert_w_std=0.3)
+    layer = W.make_layer(spec, seed=8)
+    for name in ("w_gate", "w_up", "w_down", "b_gate", "b_up", "b_down"):
+        layer[name] = np.repeat(layer[name][:1], spec.E, axis=0)
+    ref = O.layer_forward(layer, spec.k, spec.limit)
+    for t in range(spec.T):
+        _, o = brute.expert_output(layer, 0, [float(v) for v in layer["x"][t]], spec.limit)
+        np.testing.assert_allclose(ref["y"][t], o, rtol=1e-12, atol=1e-12)
+
+
+def test_router_logits_with_identity_weights():
+    """Wr = I (E = D): the logits are the activations plus the router bias."""
+    D = 6
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((7, D))
+    b = rng.standard_normal(D)
+    lg = O.router_logits(x, np.eye(D), b)
+    np.testing.assert_allclose(lg, x + b, rtol=0, atol=1e-15)
+
+
 def test_down_bias_is_weighted():
     """With zero expert weights the output is sum_j w_j * b_down[e_j]."""
     spec = W.tiny_spec(T=9, D=8, E=4, k=2, F=8, dtype="f32")
