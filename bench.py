@@ -463,8 +463,11 @@ def traffic_from_profiles(kernel, workload):
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
-    src = os.path.join(ROOT, "mixture_experts_ffn_12_b200", "csrc", "grouped_gemm.cuh")
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    # the kernel's source and its launch configuration (tile sizes live in gemm_launch.cuh)
+    h = hashlib.sha256()
+    for name in ("grouped_gemm.cuh", "gemm_launch.cuh"):
+        h.update(open(os.path.join(ROOT, "mixture_experts_ffn_12_b200", "csrc", name), "rb").read())
+    sha = h.hexdigest()[:16]
     vals = {}
     for line in open(path):
         if ":" in line and line.startswith("- "):

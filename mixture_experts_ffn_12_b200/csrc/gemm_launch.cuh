@@ -257,7 +257,7 @@ static int64_t max_row_blocks(int64_t R, int G) { return (R + kBM - 1) / kBM + G
 constexpr int kStages = 4;
 constexpr int kPairStages = 6;
 constexpr int kTNHalf = 120;     // pair tiles: each CTA holds 120 B rows (N = 240)
-constexpr int kTNGateUp = 120;   // 2 x 120 = 240 MMA columns, F = 2880 = 24 x 120
+constexpr int kTNGateUp = 128;   // 2 x 128 = 256 MMA columns (F = 2880: 23 column blocks, the last half used)
 constexpr int kTNDown = 240;     // D = 2880 = 12 x 240
 
 cudaError_t router_tc(const Launch& L, int64_t T, int D, int E, int k, const void* x, const void* w_router,
@@ -440,8 +440,12 @@ cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, i
     return launch_wm_pair<EPI_SWIGLU>(L, wg, wu, ta, tx16, a, units);
   }
   if (use_pair(R, E)) {
+    // the pair kernel's weight halves are kTNHalf rows: boxes of that height
+    CUtensorMap pg, pu;
+    if ((e = make_tmap(&pg, w.w_gate, false, D, F, E, kTNHalf)) != cudaSuccess) return e;
+    if ((e = make_tmap(&pu, w.w_up, false, D, F, E, kTNHalf)) != cudaSuccess) return e;
     const int64_t ptiles = ((R + kPairBM - 1) / kPairBM + E) * ((F + kTNHalf - 1) / kTNHalf);
-    return launch_pair<kTNHalf, EPI_SWIGLU, kPairStages>(L, ta, tg, tu, a, ptiles);
+    return launch_pair<kTNHalf, EPI_SWIGLU, kPairStages>(L, ta, pg, pu, a, ptiles);
   }
   const int64_t tiles = max_row_blocks(R, E) * ((F + kTNGateUp - 1) / kTNGateUp);
   return launch<__nv_bfloat16, kTNGateUp, 2, EPI_SWIGLU, kStages>(L, ta, tg, tu, a, tiles);
