@@ -33,6 +33,11 @@
  *    bytes [.., N, K/32] (scale 2^(s-127) for 32 consecutive elements along K),
  *    per the OCP Microscaling formats; the pages name the format "MXFP4"
  *    ("GPT-OSS 20B GGUF with MoE CPU Offloading", Model Specifications).
+ *  - Kernels are launched with programmatic dependent launch: each of the
+ *    library's kernels lets the next kernel on the stream be scheduled early and
+ *    itself waits (griddepcontrol.wait) for the preceding kernel's completion and
+ *    memory before touching any buffer, so stream order is kept for callers'
+ *    kernels and copies before and after a call.
  *  - Arguments are validated before any launch; a rejected call launches
  *    nothing and returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED /
  *    MOE_ERR_WORKSPACE.  T = 0 is a successful no-op (expert_off is zeroed
