@@ -457,17 +457,27 @@ def ctypes_ptr(h):
     return _lib.ctypes.c_void_p(int(h)).value
 
 
+def gateup_kernel_sha():
+    """Identity of the profiled gate/up kernel build: its source, the device helpers it
+    includes, and the lines of gemm_launch.cuh that fix its tile shape and ring depth."""
+    import hashlib
+    csrc = os.path.join(ROOT, "mixture_experts_ffn_12_b200", "csrc")
+    h = hashlib.sha256()
+    for name in ("grouped_gemm.cuh", "common.cuh"):
+        h.update(open(os.path.join(csrc, name), "rb").read())
+    for line in open(os.path.join(csrc, "gemm_launch.cuh")):
+        if line.startswith(("constexpr int kStages =", "constexpr int kTNGateUp =")):
+            h.update(line.encode())
+    return h.hexdigest()[:16]
+
+
 def traffic_from_profiles(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
     import hashlib
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
-    # the kernel's source and its launch configuration (tile sizes live in gemm_launch.cuh)
-    h = hashlib.sha256()
-    for name in ("grouped_gemm.cuh", "gemm_launch.cuh"):
-        h.update(open(os.path.join(ROOT, "mixture_experts_ffn_12_b200", "csrc", name), "rb").read())
-    sha = h.hexdigest()[:16]
+    sha = gateup_kernel_sha()
     vals = {}
     for line in open(path):
         if ":" in line and line.startswith("- "):

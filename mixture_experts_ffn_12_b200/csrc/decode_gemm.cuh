@@ -65,6 +65,14 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const int* unit_off, cons
   return t;
 }
 
+// Zeroes n floats (the weighted rows a K-split decode launch adds into).
+__global__ void __launch_bounds__(256) zero_f32_kernel(float* __restrict__ p, int64_t n) {
+  pdl_enter();
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = 0.0f;
+}
+
 // EPI_SWIGLU: tmW0 = W_gate, tmW1 = W_up (boxes of 64 rows); EPI_BIAS / EPI_BIAS_WSCATTER: tmW0 = W_down (128 rows).
 template <int EPI, int NTOK, int STAGES, int KBS = 1>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -160,9 +168,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = unit_off[G];
+  // EPI_BIAS_WSCATTER may split K in S ranges (units S times as many, split
+  // fastest); each range adds its weighted partial into the zeroed fp32 rows
+  const int S = (EPI == EPI_BIAS_WSCATTER && args.k_splits > 1) ? args.k_splits : 1;
+  const int total = unit_off[G] * S;
+  const int per_split = (KSTEP_STAGES + S - 1) / S;
 
-  auto unit = [&](int u) { return decode_unit(u, unit_off, goff, G, FB, FBW, NTOK); };
+  auto unit = [&](int u) { return decode_unit(u / S, unit_off, goff, G, FB, FBW, NTOK); };
+  auto stage_range = [&](int u, int& b, int& e) {
+    b = (u % S) * per_split;
+    e = min(KSTEP_STAGES, b + per_split);
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -173,7 +189,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
         const UnitInfo ui = unit(u);
-        for (int ks = 0; ks < KSTEP_STAGES; ++ks) {
+        int ks0, ks1;
+        stage_range(u, ks0, ks1);
+        for (int ks = ks0; ks < ks1; ++ks) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], tx_bytes);
 #pragma unroll
@@ -216,7 +234,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, lim)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * NTOK);
-        for (int ks = 0; ks < KSTEP_STAGES; ++ks) {
+        int ks0, ks1;
+        stage_range(u, ks0, ks1);
+        for (int ks = ks0; ks < ks1; ++ks) {
           if (!mbar_wait(&full[s], ph, abort_flag, lim)) { ok = false; break; }
           tc_fence_after();
           const uint32_t stage_addr = smem_u32(smem + s * LY::STAGE_BYTES);
@@ -227,7 +247,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < KSTEPS; ++kk)
               tc_mma<false>(d_tmem, sw128_kmajor_desc(w_addr + kk * 32), sw128_kmajor_desc(x_addr + kk * 32), idesc,
-                            (ks | b | kk) != 0 ? 1u : 0u);
+                            (ks != ks0 || b != 0 || kk != 0) ? 1u : 0u);
           }
           tc_commit(&empty[s]);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -305,7 +325,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 flag_error(DEVERR_BOUNDS);
                 continue;
               }
-              static_cast<float*>(args.out)[static_cast<size_t>(slot) * args.ldo + d] = args.topk_w[slot] * (v[c] + b);
+              float* dst = static_cast<float*>(args.out) + static_cast<size_t>(slot) * args.ldo + d;
+              if (S == 1) {
+                *dst = args.topk_w[slot] * (v[c] + b);
+              } else {
+                // the K ranges add into zeroed memory; the first carries the bias.  With
+                // two ranges the sum is the same whichever lands first (0 + x + y = x + y)
+                atomicAdd(dst, args.topk_w[slot] * (v[c] + (u % S == 0 ? b : 0.0f)));
+              }
             } else {
               static_cast<T*>(args.out)[static_cast<size_t>(row) * args.ldo + d] = __float2bfloat16_rn(v[c] + b);
             }

@@ -496,7 +496,19 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
     if ((e = make_tmap(&wd, w.w_down, false, F, D, E, 128)) != cudaSuccess) return e;
     if ((e = make_tmap(&th, h, false, F, R, 0, kDecTok)) != cudaSuccess) return e;
     const int64_t units = (std::min<int64_t>(E, R) + R / kDecTok) * ((D + 127) / 128);
-    if (slot_of_row != nullptr) return launch_decode<EPI_BIAS_WSCATTER>(L, wd, wd, th, a, units);
+    if (slot_of_row != nullptr) {
+      if (units <= L.num_sms) {
+        // fewer units than SMs (T = 1: 4 experts x 23 feature blocks): split K in two,
+        // each half adding its weighted partial into the zeroed fp32 rows
+        const int64_t n = R * static_cast<int64_t>(D);
+        pdl_launch(zero_f32_kernel, dim3(static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 4 * L.num_sms))),
+                   dim3(256), 0, L.stream, static_cast<float*>(out), n);
+        count_launch();
+        a.k_splits = 2;
+        return launch_decode<EPI_BIAS_WSCATTER>(L, wd, wd, th, a, 2 * units);
+      }
+      return launch_decode<EPI_BIAS_WSCATTER>(L, wd, wd, th, a, units);
+    }
     return launch_decode<EPI_BIAS>(L, wd, wd, th, a, units);
   }
   if (gemm_kind(R, E, true) == GK_WM_PAIR) {
