@@ -284,6 +284,43 @@ def test_unrouted_expert_contributes_nothing():
     np.testing.assert_array_equal(ref2["y"], ref["y"])
 
 
+def test_swiglu_is_odd_in_up_and_flat_beyond_the_limits():
+    """h(g, -u) = -h(g, u) (the up clip is symmetric), h is constant in u beyond +/-L and
+    in g beyond L, and scales linearly in u inside the clip range."""
+    rng = np.random.default_rng(10)
+    g = rng.uniform(-3, 10, 200)
+    u = rng.uniform(-10, 10, 200)
+    L = 7.0
+    np.testing.assert_array_equal(O.clipped_swiglu(g, -u, L), -O.clipped_swiglu(g, u, L))
+    np.testing.assert_array_equal(O.clipped_swiglu(g, np.full_like(u, 9.0), L), O.clipped_swiglu(g, np.full_like(u, L), L))
+    np.testing.assert_array_equal(O.clipped_swiglu(np.full_like(g, 12.0), u, L), O.clipped_swiglu(np.full_like(g, L), u, L))
+    inside = np.abs(u) < L / 2
+    np.testing.assert_allclose(O.clipped_swiglu(g[inside], 2 * u[inside], L), 2 * O.clipped_swiglu(g[inside], u[inside], L),
+                               rtol=1e-15, atol=0)
+
+
+def test_mxfp4_scale_step_doubles_every_weight():
+    """Raising every E8M0 byte by one doubles every dequantised weight exactly."""
+    rng = np.random.default_rng(11)
+    q = rng.integers(0, 256, size=(3, 5, 32), dtype=np.uint8)        # [E, N, K/2] = 64 codes per row
+    s = rng.integers(100, 140, size=(3, 5, 2), dtype=np.uint8)       # two 32-element blocks per row
+    np.testing.assert_array_equal(O.mxfp4_dequant(q, s + 1), 2.0 * O.mxfp4_dequant(q, s))
+
+
+def test_output_is_linear_in_the_down_projection():
+    """Doubling W_down and b_down doubles y exactly (routing and h are untouched)."""
+    spec = W.tiny_spec(T=10, D=16, E=4, k=2, F=24, dtype="f32", expert_w_std=0.3)
+    layer = W.make_layer(spec, seed=12)
+    ref = O.layer_forward(layer, spec.k, spec.limit)
+    l2 = dict(layer)
+    l2["w_down"] = 2.0 * layer["w_down"]
+    l2["b_down"] = 2.0 * layer["b_down"]
+    ref2 = O.layer_forward(l2, spec.k, spec.limit)
+    np.testing.assert_array_equal(ref2["ids"], ref["ids"])
+    np.testing.assert_array_equal(ref2["h"], ref["h"])
+    np.testing.assert_allclose(ref2["y"], 2.0 * ref["y"], rtol=1e-14, atol=0)
+
+
 def test_identical_experts_give_the_dense_mlp():
     """If every expert has the same weights and biases, routing cannot matter: the softmax
     weights sum to 1, so every token's output is that one dense MLP's output (a scalar
