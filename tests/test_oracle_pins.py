@@ -385,6 +385,55 @@ def test_pins_catch_planted_dispatch_mistake():
     assert unstable.tolist() != sor
 
 
+def test_pins_catch_planted_layer_mistakes():
+    """Plausible mistakes in the layer arithmetic, each written out as a variant of the
+    layer (numpy, fp64), all disagree with the scalar-loop layer on a tiny case where the
+    oracle itself agrees to 1e-12: softmax over all experts, selection of the smallest
+    logits, a dropped down bias, an unweighted down bias, a transposed gate weight, gate
+    and up swapped, and an unnormalised routing weight."""
+    spec = W.tiny_spec(T=6, D=12, E=5, k=2, F=12, dtype="f32", expert_w_std=0.4, router_w_std=0.5)
+    layer = W.make_layer(spec, seed=13, logits_fn=_logits_fn)
+    L, a = spec.limit, 1.702
+    x = O.decode(layer["x"])
+    lg = O.router_logits(layer["x"], layer["w_router"], layer["b_router"])
+    Wg, Wu, Wd = (O.expert_weights(layer, n) for n in ("gate", "up", "down"))
+    bg, bu, bd = (O.decode(layer[f"b_{n}"]) for n in ("gate", "up", "down"))
+
+    def layer_y(select="top", weights="softmax_k", bias="weighted", gate_t=False, swap=False):
+        ys = np.zeros((spec.T, spec.D))
+        for t in range(spec.T):
+            order = np.argsort(-lg[t], kind="stable") if select == "top" else np.argsort(lg[t], kind="stable")
+            ids = order[:spec.k]
+            if weights == "softmax_k":
+                e = np.exp(lg[t, ids] - lg[t, ids].max()); w = e / e.sum()
+            elif weights == "softmax_all":
+                e = np.exp(lg[t] - lg[t].max()); w = (e / e.sum())[ids]
+            else:
+                w = np.exp(lg[t, ids] - lg[t, ids].max())
+            for j, ex in enumerate(ids):
+                wg = Wg[ex].T if gate_t else Wg[ex]
+                g = wg @ x[t] + bg[ex]
+                u = Wu[ex] @ x[t] + bu[ex]
+                if swap:
+                    g, u = u, g
+                h = O.clipped_swiglu(g, u, L, a)
+                o = Wd[ex] @ h
+                if bias == "weighted":
+                    ys[t] += w[j] * (o + bd[ex])
+                elif bias == "unweighted":
+                    ys[t] += w[j] * o + bd[ex]
+                else:
+                    ys[t] += w[j] * o
+        return ys
+
+    want = np.array([brute.layer_token(layer, t, spec.k, L)["y"] for t in range(spec.T)])
+    np.testing.assert_allclose(O.layer_forward(layer, spec.k, L)["y"], want, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(layer_y(), want, rtol=1e-12, atol=1e-12)
+    for kw in (dict(weights="softmax_all"), dict(select="bottom"), dict(bias="none"), dict(bias="unweighted"),
+               dict(gate_t=True), dict(swap=True), dict(weights="unnormalised")):
+        assert not np.allclose(layer_y(**kw), want, rtol=1e-6, atol=1e-9), kw
+
+
 # --------------------------------------------------------------------------- #
 # input recipes
 # --------------------------------------------------------------------------- #
