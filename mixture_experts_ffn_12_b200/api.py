@@ -59,6 +59,116 @@ def _p(t: Optional[torch.Tensor]):
     return ctypes.c_void_p(t.data_ptr())
 
 
+# --------------------------------------------------------------------------- #
+# argument checks: the C ABI sees pointers only, so shapes and dtypes are checked
+# here, against the layouts include/moe.h documents, before any pointer is passed
+# (a bf16 buffer passed where fp32 is declared would be read past its end).
+# These checks touch no device and run on CPU tensors too.
+# --------------------------------------------------------------------------- #
+def _want(name: str, t: Optional[torch.Tensor], shape, dtype: torch.dtype,
+          device: Optional[torch.device] = None) -> None:
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _rows(name: str, t: Optional[torch.Tensor]) -> int:
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dim() == 0:
+        raise ValueError(f"{name} must have a leading token dimension")
+    return int(t.shape[0])
+
+
+def check_expert_weights(cfg: MoeConfig, w: "ExpertWeights", device: Optional[torch.device] = None) -> None:
+    """Dense: W_g, W_u [E, F, D], W_d [E, D, F] in the layer dtype.  MXFP4: packed E2M1
+    codes [E, F, D/2], [E, F, D/2], [E, D, F/2] and E8M0 scales [E, F, D/32], [E, F, D/32],
+    [E, D, F/32], all uint8.  Biases [E, F], [E, F], [E, D] in the layer dtype."""
+    D, F, E = cfg.hidden_size, cfg.intermediate_size, cfg.num_local_experts
+    dt = torch_dtype(cfg)
+    if cfg.wfmt == _lib.MOE_W_MXFP4:
+        if D % 32 or F % 32:
+            raise ValueError(f"MXFP4 weights need D and F divisible by 32 (D={D}, F={F})")
+        _want("w_gate", w.w_gate, (E, F, D // 2), torch.uint8, device)
+        _want("w_up", w.w_up, (E, F, D // 2), torch.uint8, device)
+        _want("w_down", w.w_down, (E, D, F // 2), torch.uint8, device)
+        _want("s_gate", w.s_gate, (E, F, D // 32), torch.uint8, device)
+        _want("s_up", w.s_up, (E, F, D // 32), torch.uint8, device)
+        _want("s_down", w.s_down, (E, D, F // 32), torch.uint8, device)
+    else:
+        _want("w_gate", w.w_gate, (E, F, D), dt, device)
+        _want("w_up", w.w_up, (E, F, D), dt, device)
+        _want("w_down", w.w_down, (E, D, F), dt, device)
+    _want("b_gate", w.b_gate, (E, F), dt, device)
+    _want("b_up", w.b_up, (E, F), dt, device)
+    _want("b_down", w.b_down, (E, D), dt, device)
+
+
+def check_router_args(cfg: MoeConfig, x, w_router, b_router, topk_ids=None, topk_w=None) -> int:
+    """x [T, D], W_r [E, D], b_r [E] in the layer dtype; topk_ids [T, k] int32 and
+    topk_w [T, k] fp32 when given.  Returns T."""
+    D, E, k = cfg.hidden_size, cfg.num_local_experts, cfg.num_experts_per_tok
+    dt = torch_dtype(cfg)
+    T = _rows("x", x)
+    _want("x", x, (T, D), dt)
+    _want("w_router", w_router, (E, D), dt, x.device)
+    _want("b_router", b_router, (E,), dt, x.device)
+    if topk_ids is not None:
+        _want("topk_ids", topk_ids, (T, k), torch.int32, x.device)
+    if topk_w is not None:
+        _want("topk_w", topk_w, (T, k), torch.float32, x.device)
+    return T
+
+
+def check_permute_args(cfg: MoeConfig, topk_ids, x=None) -> int:
+    """topk_ids [T, k] int32; x [T, D] in the layer dtype when given.  Returns T."""
+    T = _rows("topk_ids", topk_ids)
+    _want("topk_ids", topk_ids, (T, cfg.num_experts_per_tok), torch.int32)
+    if x is not None:
+        _want("x", x, (T, cfg.hidden_size), torch_dtype(cfg), topk_ids.device)
+    return T
+
+
+def check_expert_ffn_args(cfg: MoeConfig, x_perm, expert_off, weights: "ExpertWeights") -> int:
+    """x_perm [R, D] in the layer dtype with R = T·k; expert_off [E+1] int32.  Returns T."""
+    R, k = _rows("x_perm", x_perm), cfg.num_experts_per_tok
+    if R % k:
+        raise ValueError(f"x_perm has {R} rows, not a multiple of k = {k}")
+    _want("x_perm", x_perm, (R, cfg.hidden_size), torch_dtype(cfg))
+    _want("expert_off", expert_off, (cfg.num_local_experts + 1,), torch.int32, x_perm.device)
+    check_expert_weights(cfg, weights, x_perm.device)
+    return R // k
+
+
+def check_combine_args(cfg: MoeConfig, y_perm, row_of_slot, topk_w) -> int:
+    """y_perm [T·k, D] in the layer dtype; row_of_slot [T, k] int32; topk_w [T, k] fp32.  Returns T."""
+    k = cfg.num_experts_per_tok
+    T = _rows("row_of_slot", row_of_slot)
+    _want("row_of_slot", row_of_slot, (T, k), torch.int32)
+    _want("y_perm", y_perm, (T * k, cfg.hidden_size), torch_dtype(cfg), row_of_slot.device)
+    _want("topk_w", topk_w, (T, k), torch.float32, row_of_slot.device)
+    return T
+
+
+def check_layer_args(cfg: MoeConfig, x, w_router, b_router, weights: Optional["ExpertWeights"], y=None,
+                     topk_ids=None, topk_w=None) -> int:
+    """The router's arguments, the expert weights (skipped when None: already checked)
+    and y [T, D] in the layer dtype when given.  Returns T."""
+    T = check_router_args(cfg, x, w_router, b_router, topk_ids, topk_w)
+    if weights is not None:
+        check_expert_weights(cfg, weights, x.device)
+    if y is not None:
+        _want("y", y, (T, cfg.hidden_size), torch_dtype(cfg), x.device)
+    return T
+
+
 def _stream(device: torch.device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
@@ -99,24 +209,33 @@ def expert_weights_from(d: Dict[str, torch.Tensor]) -> ExpertWeights:
 
 
 # --------------------------------------------------------------------------- #
-# the five calls
+# the five calls (each on torch's current stream of the tensors' device)
 # --------------------------------------------------------------------------- #
+def _size(n: int, what: str) -> int:
+    if n == _lib.SIZE_INVALID:
+        raise MoeError(_lib.MOE_ERR_INVALID_ARG, what)
+    return n
+
+
 def router_topk(cfg: MoeConfig, x: torch.Tensor, w_router: torch.Tensor, b_router: torch.Tensor,
                 topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None
                 ) -> Tuple[torch.Tensor, torch.Tensor]:
-    T, k = x.shape[0], cfg.num_experts_per_tok
+    T = check_router_args(cfg, x, w_router, b_router, topk_ids, topk_w)
+    k = cfg.num_experts_per_tok
     if topk_ids is None:
         topk_ids = torch.empty((T, k), dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty((T, k), dtype=torch.float32, device=x.device)
-    _check(_lib.load().moe_router_topk(ctypes.byref(cfg), T, _p(x), _p(w_router), _p(b_router), _p(topk_ids),
-                                       _p(topk_w), _stream(x.device)), "moe_router_topk")
+    with torch.cuda.device(x.device):
+        _check(_lib.load().moe_router_topk(ctypes.byref(cfg), T, _p(x), _p(w_router), _p(b_router), _p(topk_ids),
+                                           _p(topk_w), _stream(x.device)), "moe_router_topk")
     return topk_ids, topk_w
 
 
 def permute(cfg: MoeConfig, topk_ids: torch.Tensor, x: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+    T = check_permute_args(cfg, topk_ids, x)
     L = _lib.load()
-    T, k, dev = topk_ids.shape[0], cfg.num_experts_per_tok, topk_ids.device
+    k, dev = cfg.num_experts_per_tok, topk_ids.device
     R = T * k
     out = dict(
         expert_off=torch.empty(cfg.num_local_experts + 1, dtype=torch.int32, device=dev),
@@ -124,57 +243,63 @@ def permute(cfg: MoeConfig, topk_ids: torch.Tensor, x: Optional[torch.Tensor] = 
         slot_of_row=torch.empty(R, dtype=torch.int32, device=dev),
     )
     out["x_perm"] = None if x is None else torch.empty((R, cfg.hidden_size), dtype=x.dtype, device=dev)
-    nws = L.moe_permute_workspace_size(ctypes.byref(cfg), T)
+    nws = _size(L.moe_permute_workspace_size(ctypes.byref(cfg), T), "moe_permute_workspace_size")
     ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
-    _check(L.moe_permute(ctypes.byref(cfg), T, _p(topk_ids), _p(x), _p(out["expert_off"]), _p(out["row_of_slot"]),
-                         _p(out["slot_of_row"]), _p(out["x_perm"]), _p(ws), ws.numel(), _stream(dev)),
-           "moe_permute")
+    with torch.cuda.device(dev):
+        _check(L.moe_permute(ctypes.byref(cfg), T, _p(topk_ids), _p(x), _p(out["expert_off"]),
+                             _p(out["row_of_slot"]), _p(out["slot_of_row"]), _p(out["x_perm"]), _p(ws), ws.numel(),
+                             _stream(dev)), "moe_permute")
     return out
 
 
 def expert_ffn(cfg: MoeConfig, x_perm: torch.Tensor, expert_off: torch.Tensor, weights: ExpertWeights
                ) -> Tuple[torch.Tensor, torch.Tensor]:
+    T = check_expert_ffn_args(cfg, x_perm, expert_off, weights)
     L = _lib.load()
     R, dev = x_perm.shape[0], x_perm.device
-    T = R // cfg.num_experts_per_tok
     dt = torch_dtype(cfg)
     h = torch.empty((R, cfg.intermediate_size), dtype=dt, device=dev)
     y_perm = torch.empty((R, cfg.hidden_size), dtype=dt, device=dev)
-    nws = L.moe_expert_ffn_workspace_size(ctypes.byref(cfg), T)
+    nws = _size(L.moe_expert_ffn_workspace_size(ctypes.byref(cfg), T), "moe_expert_ffn_workspace_size")
     ws = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
     ws_struct = weights.c_struct()
-    _check(L.moe_expert_ffn(ctypes.byref(cfg), T, _p(x_perm), _p(expert_off), ctypes.byref(ws_struct), _p(h),
-                            _p(y_perm), _p(ws), nws, _stream(dev)), "moe_expert_ffn")
+    with torch.cuda.device(dev):
+        _check(L.moe_expert_ffn(ctypes.byref(cfg), T, _p(x_perm), _p(expert_off), ctypes.byref(ws_struct), _p(h),
+                                _p(y_perm), _p(ws), nws, _stream(dev)), "moe_expert_ffn")
     return h, y_perm
 
 
 def combine(cfg: MoeConfig, y_perm: torch.Tensor, row_of_slot: torch.Tensor, topk_w: torch.Tensor) -> torch.Tensor:
-    T, dev = row_of_slot.shape[0], y_perm.device
+    T = check_combine_args(cfg, y_perm, row_of_slot, topk_w)
+    dev = y_perm.device
     y = torch.empty((T, cfg.hidden_size), dtype=y_perm.dtype, device=dev)
-    _check(_lib.load().moe_combine(ctypes.byref(cfg), T, _p(y_perm), _p(row_of_slot), _p(topk_w), _p(y),
-                                   _stream(dev)), "moe_combine")
+    with torch.cuda.device(dev):
+        _check(_lib.load().moe_combine(ctypes.byref(cfg), T, _p(y_perm), _p(row_of_slot), _p(topk_w), _p(y),
+                                       _stream(dev)), "moe_combine")
     return y
 
 
 def workspace_size(cfg: MoeConfig, T: int) -> int:
-    n = _lib.load().moe_workspace_size(ctypes.byref(cfg), T)
-    if n == _lib.SIZE_INVALID:
-        raise MoeError(_lib.MOE_ERR_INVALID_ARG, "moe_workspace_size")
-    return n
+    return _size(_lib.load().moe_workspace_size(ctypes.byref(cfg), T), "moe_workspace_size")
 
 
 def layer_forward(cfg: MoeConfig, x: torch.Tensor, w_router: torch.Tensor, b_router: torch.Tensor,
                   weights: ExpertWeights, y: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-                  topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None) -> torch.Tensor:
-    T, dev = x.shape[0], x.device
+                  topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                  _weights_checked: bool = False) -> torch.Tensor:
+    T = check_layer_args(cfg, x, w_router, b_router, None if _weights_checked else weights, y, topk_ids, topk_w)
+    dev = x.device
     if y is None:
         y = torch.empty((T, cfg.hidden_size), dtype=x.dtype, device=dev)
     if ws is None:
         ws = torch.empty(max(workspace_size(cfg, T), 16), dtype=torch.uint8, device=dev)
+    elif ws.device != dev:
+        raise ValueError(f"ws is on {ws.device}, expected {dev}")
     wst = weights.c_struct()
-    _check(_lib.load().moe_layer_forward(ctypes.byref(cfg), T, _p(x), _p(w_router), _p(b_router),
-                                         ctypes.byref(wst), _p(y), _p(topk_ids), _p(topk_w), _p(ws), ws.numel(),
-                                         _stream(dev)), "moe_layer_forward")
+    with torch.cuda.device(dev):
+        _check(_lib.load().moe_layer_forward(ctypes.byref(cfg), T, _p(x), _p(w_router), _p(b_router),
+                                             ctypes.byref(wst), _p(y), _p(topk_ids), _p(topk_w), _p(ws),
+                                             ws.numel() * ws.element_size(), _stream(dev)), "moe_layer_forward")
     return y
 
 
@@ -184,7 +309,9 @@ def last_device_error() -> int:
 
 
 def set_expert_gemm_variant(variant: int) -> None:
-    """0 = by size, 1 = single-CTA tiles, 2 = CTA-pair tiles (bf16 expert GEMMs)."""
+    """Expert-GEMM kernel choice for bf16 dense weights: 0 = by size (the default), 1 = single-CTA
+    128-row tiles, 2 = CTA-pair 256-row tiles, 3 = the weight-stationary decode kernel,
+    4 = CTA pairs with the weights in M.  Process-wide; MXFP4 layers ignore it."""
     _check(_lib.load().moe_set_expert_gemm_variant(variant), "moe_set_expert_gemm_variant")
 
 
@@ -196,6 +323,8 @@ class MoELayer:
     """A GPT-OSS MoE FFN layer resident on one GPU: weights, config and a reusable workspace."""
 
     def __init__(self, cfg: MoeConfig, w_router: torch.Tensor, b_router: torch.Tensor, experts: ExpertWeights):
+        _check(_lib.load().moe_config_check(ctypes.byref(cfg)), "moe_config_check")
+        check_expert_weights(cfg, experts, w_router.device)
         self.cfg, self.w_router, self.b_router, self.experts = cfg, w_router, b_router, experts
         self._ws: Optional[torch.Tensor] = None
 
@@ -207,7 +336,8 @@ class MoELayer:
 
     def __call__(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, topk_ids=None, topk_w=None) -> torch.Tensor:
         return layer_forward(self.cfg, x, self.w_router, self.b_router, self.experts, y=y,
-                             ws=self.workspace(x.shape[0]), topk_ids=topk_ids, topk_w=topk_w)
+                             ws=self.workspace(_rows("x", x)), topk_ids=topk_ids, topk_w=topk_w,
+                             _weights_checked=True)
 
     def graphed(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, topk_ids=None, topk_w=None):
         """Capture one forward on these fixed buffers into a CUDA graph; returns (replay, y).
@@ -224,7 +354,7 @@ class MoELayer:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             layer_forward(self.cfg, x, self.w_router, self.b_router, self.experts, y=y, ws=ws,
-                          topk_ids=topk_ids, topk_w=topk_w)
+                          topk_ids=topk_ids, topk_w=topk_w, _weights_checked=True)
         return g.replay, y
 
     def run_host_batches(self, xs_host, ys_host) -> None:
