@@ -12,8 +12,12 @@ Two levels:
   * ``brute``      (O0): pure-Python scalar loops, for tiny inputs only; it is
     what O1 is pinned against.
 
+``glm_moe`` is the O1 oracle of the layer's GLM4-MoE-Lite variant (sigmoid
+router with a selection-only correction bias, SiLU experts, a shared expert);
+``brute`` holds its scalar-loop counterpart.
+
 Every function is pinned by ``tests/test_oracle_pins.py`` (brute force, closed
 forms, invariants, hand-worked values in ``tests/golden/``).  No function here
 is "parity unpinned".
 """
-from . import moe_oracle, brute  # noqa: F401
+from . import moe_oracle, brute, glm_moe  # noqa: F401

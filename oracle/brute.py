@@ -8,13 +8,17 @@ dispatch and weighted combine from "Ollama glm4_moe_lite.go").
 
 Top-k here is found by enumerating every k-subset of experts, not by sorting;
 the dispatch permutation by counting, not by a library sort.
+
+The last section does the same for the GLM4-MoE-Lite variant of the layer
+(sigmoid router with a selection-only correction bias, SiLU experts without
+biases, a shared expert), pinning ``glm_moe``.
 """
 from __future__ import annotations
 
 import itertools
 import math
 import struct
-from typing import Dict, List, Sequence, Tuple
+from typing import Dict, List, Optional, Sequence, Tuple
 
 
 def bf16_value(bits: int) -> float:
@@ -175,3 +179,70 @@ def layer_token(layer, t: int, k: int, limit: float, alpha: float = 1.702) -> Di
         for d in range(D):
             y[d] += w[j] * o[d]
     return dict(logits=lg, ids=ids, w=w, h=hs, y=y)
+
+
+# --------------------------------------------------------------------------- #
+# GLM4-MoE-Lite variant ("Ollama glm4_moe_lite.go": MoEGate.Forward,
+# SwitchMLP.Forward, SharedExperts.Forward, MoE.Forward), by scalar loops
+# --------------------------------------------------------------------------- #
+def silu(z: float) -> float:
+    return z * sigmoid(z)
+
+
+def glm_route_bruteforce(logits: Sequence[float], k: int, correction: Optional[Sequence[float]],
+                         norm_topk_prob: bool, routed_scaling_factor: float) -> Tuple[List[int], List[float]]:
+    """Experts chosen by enumerating k-subsets on the corrected sigmoid scores.
+
+    The chosen subset is the one whose every member beats every non-member
+    (larger corrected score, equal scores: lower index); the weights are the
+    uncorrected scores of the chosen experts, normalised by their sum when
+    k > 1 and ``norm_topk_prob``, then scaled.
+    """
+    E = len(logits)
+    score = [sigmoid(v) for v in logits]
+    sel = [score[e] + (correction[e] if correction is not None else 0.0) for e in range(E)]
+    ids, _ = topk_bruteforce(sel, k)      # subset enumeration, ordered by a selection pass
+    w = [score[e] for e in ids]
+    if k > 1 and norm_topk_prob:
+        z = 0.0
+        for v in w:
+            z += v
+        w = [v / z for v in w]
+    return ids, [v * routed_scaling_factor for v in w]
+
+
+def silu_mlp_row(x: Sequence[float], wg_rows, wu_rows, wd_rows) -> List[float]:
+    """o = W_d (SiLU(W_g x) * (W_u x)) for one activation row; weights given as row lists."""
+    h = [silu(dot(x, wg_rows[f])) * dot(x, wu_rows[f]) for f in range(len(wg_rows))]
+    return [dot(h, wd_rows[d]) for d in range(len(wd_rows))]
+
+
+def glm_layer_token(layer, t: int, k: int, norm_topk_prob: bool, routed_scaling_factor: float) -> Dict[str, list]:
+    """The GLM4-MoE-Lite layer for token t, by scalar loops."""
+    x = [value(v) for v in layer["x"][t]]
+    E = layer["w_router"].shape[0]
+    lg = []
+    for e in range(E):
+        v = dot(x, [value(q) for q in layer["w_router"][e]])
+        if layer.get("b_router") is not None:
+            v += value(layer["b_router"][e])
+        lg.append(v)
+    corr = layer.get("e_score_correction_bias")
+    corr = None if corr is None else [value(v) for v in corr]
+    ids, w = glm_route_bruteforce(lg, k, corr, norm_topk_prob, routed_scaling_factor)
+    D = layer["w_down"].shape[1]
+    y = [0.0] * D
+    for j in range(k):
+        e = ids[j]
+        o = silu_mlp_row(x, [[value(q) for q in r] for r in layer["w_gate"][e]],
+                         [[value(q) for q in r] for r in layer["w_up"][e]],
+                         [[value(q) for q in r] for r in layer["w_down"][e]])
+        for d in range(D):
+            y[d] += w[j] * o[d]
+    if "ws_gate" in layer:
+        o = silu_mlp_row(x, [[value(q) for q in r] for r in layer["ws_gate"]],
+                         [[value(q) for q in r] for r in layer["ws_up"]],
+                         [[value(q) for q in r] for r in layer["ws_down"]])
+        for d in range(D):
+            y[d] += o[d]
+    return dict(logits=lg, ids=ids, w=w, y=y)

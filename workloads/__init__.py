@@ -21,6 +21,11 @@ Parameter names follow the GPT-OSS weight map on the MaxText page
 each with a bias); the layer sizes follow the GPT-OSS Config
 (hidden_size, num_local_experts, num_experts_per_tok, swiglu_limit) and the
 GPT-OSS 20B model card (32 experts, 4 active per token; MXFP4 expert weights).
+
+``GlmLayerSpec`` / ``make_glm_layer`` are the recipes of the layer's GLM4-MoE-Lite
+variant ("Ollama glm4_moe_lite.go"): a router without bias plus an
+``e_score_correction_bias`` [E], expert weights without biases, and a shared
+expert ws_gate / ws_up [F_shared, D], ws_down [D, F_shared].
 """
 from __future__ import annotations
 
@@ -232,3 +237,84 @@ def tiny_spec(T: int, D: int, E: int, k: int, F: int, dtype: str = "f32", wfmt: 
                      dtype=dtype, wfmt=wfmt, router_w_std=kw.pop("router_w_std", 0.05),
                      router_b=router_b, expert_w_std=kw.pop("expert_w_std", 0.02),
                      cfg_id=cfg_id, **kw)
+
+
+# --------------------------------------------------------------------------- #
+# GLM4-MoE-Lite variant of the layer ("Ollama glm4_moe_lite.go": Config,
+# MoEGate, SwitchMLP, SharedExperts).  The page gives the config field names
+# but no sizes, so the variant's layers take the GPT-OSS-shaped sizes above.
+# --------------------------------------------------------------------------- #
+@dataclasses.dataclass(frozen=True)
+class GlmLayerSpec:
+    """One synthetic GLM4-MoE-Lite-style layer: sigmoid router with a selection-only
+    correction bias, SiLU experts without biases, an optional shared expert."""
+
+    name: str
+    T: int
+    D: int                 # hidden_size
+    E: int                 # n_routed_experts
+    k: int                 # num_experts_per_tok
+    F: int                 # moe_intermediate_size
+    F_shared: int          # intermediate size of the shared expert (0: no shared expert)
+    dtype: str             # "f32" or "bf16"
+    norm_topk_prob: bool = True
+    routed_scaling_factor: float = 2.5
+    x_std: float = 1.0
+    router_w_std: Optional[float] = None       # None -> 1/sqrt(D)
+    correction_b_std: Optional[float] = 0.1    # None: no e_score_correction_bias
+    expert_w_std: Optional[float] = None       # None -> 1/sqrt(fan_in)
+    cfg_id: int = 300
+
+    @property
+    def R(self) -> int:
+        return self.T * self.k
+
+
+_S_CB, _S_SG, _S_SU, _S_SD = 10, 11, 12, 13
+
+
+def make_glm_layer(spec: GlmLayerSpec, seed: int = 0,
+                   scores_fn: Optional[Callable[[Dict[str, np.ndarray]], np.ndarray]] = None,
+                   min_gap: float = 1e-3, max_redraw: int = 64) -> Dict[str, np.ndarray]:
+    """Draw every tensor of a variant layer.
+
+    x [T, D], w_router [E, D], e_score_correction_bias [E] (when
+    ``correction_b_std`` is set), w_gate / w_up [E, F, D], w_down [E, D, F], and
+    for the shared expert ws_gate / ws_up [F_shared, D], ws_down [D, F_shared].
+    ``scores_fn(layer) -> float64 [T, E]`` (the scores the experts are chosen by)
+    turns on the near-tie rejection, as for ``make_layer``.
+    """
+    T, D, E, F = spec.T, spec.D, spec.E, spec.F
+    out: Dict[str, np.ndarray] = {}
+    out["x"] = _normal(_rng(spec, seed, _S_X, T), (T, D), spec.x_std, spec.dtype)
+    wr_std = spec.router_w_std if spec.router_w_std is not None else 1.0 / math.sqrt(D)
+    out["w_router"] = _normal(_rng(spec, seed, _S_WR), (E, D), wr_std, spec.dtype)
+    if spec.correction_b_std is not None:
+        out["e_score_correction_bias"] = _normal(_rng(spec, seed, _S_CB), (E,), spec.correction_b_std, spec.dtype)
+    for name, stream, n, kdim in (("gate", _S_WG, F, D), ("up", _S_WU, F, D), ("down", _S_WD, D, F)):
+        std = spec.expert_w_std if spec.expert_w_std is not None else 1.0 / math.sqrt(kdim)
+        w = np.empty((E, n, kdim), dtype=np.uint16 if spec.dtype == "bf16" else np.float32)
+        for e in range(E):
+            w[e] = _normal(_rng(spec, seed, stream, e), (n, kdim), std, spec.dtype)
+        out[f"w_{name}"] = w
+    if spec.F_shared > 0:
+        Fs = spec.F_shared
+        for name, stream, n, kdim in (("gate", _S_SG, Fs, D), ("up", _S_SU, Fs, D), ("down", _S_SD, D, Fs)):
+            std = spec.expert_w_std if spec.expert_w_std is not None else 1.0 / math.sqrt(kdim)
+            out[f"ws_{name}"] = _normal(_rng(spec, seed, stream), (n, kdim), std, spec.dtype)
+    if scores_fn is not None and spec.k < E:
+        _reject_near_ties(spec, seed, out, scores_fn, min_gap, max_redraw)
+    return out
+
+
+def glm_tiny_spec(T: int, D: int, E: int, k: int, F: int, F_shared: int, dtype: str = "f32",
+                  cfg_id: int = 310, **kw) -> GlmLayerSpec:
+    """Small variant layers with the tiny-config value laws."""
+    return GlmLayerSpec(name=f"glm_tiny_T{T}_D{D}_E{E}_k{k}_F{F}_S{F_shared}_{dtype}", T=T, D=D, E=E, k=k, F=F,
+                        F_shared=F_shared, dtype=dtype, router_w_std=kw.pop("router_w_std", 0.05),
+                        expert_w_std=kw.pop("expert_w_std", 0.02), cfg_id=cfg_id, **kw)
+
+
+GLM_GPTOSS20B_SHAPE = GlmLayerSpec(
+    name="glm_variant_gptoss20b_shape", T=4096, D=2880, E=32, k=4, F=2880, F_shared=2880, dtype="bf16",
+    cfg_id=320)
