@@ -242,6 +242,61 @@ MOE_API uint64_t moe_launch_count(void);
  * moe_last_device_error then reports. */
 MOE_API void moe_set_wait_limit_ns(uint64_t ns);
 
+/* ------------------------------------------------------------------------ *
+ * The GLM4-MoE-Lite variant of the layer ("Ollama glm4_moe_lite.go":
+ * MoEGate.Forward, SwitchMLP.Forward, SharedExperts.Forward, MoE.Forward):
+ *   l[t,e]  = x[t] . Wr[e]                               gate linear, no bias
+ *   s[t,e]  = sigmoid(l[t,e])
+ *   S_t     = the k largest s[t,e] + c[e] (c = e_score_correction_bias, zero
+ *             when absent), listed by descending value, ties -> lower index
+ *   w[t,j]  = s[t,S_t[j]] / (sum_i s[t,S_t[i]] if k > 1 and norm_topk_prob,
+ *             else 1), times routed_scaling_factor
+ *   o_e     = (SiLU(x[t] Wg[e]^T) * (x[t] Wu[e]^T)) Wd[e]^T   (no biases, no clip)
+ *   y[t]    = sum_j w[t,j] o_{S_t[j]} + shared(x[t]),
+ *             shared(x) = (SiLU(x Wsg^T) * (x Wsu^T)) Wsd^T (n_shared_experts > 0)
+ * It takes the same moe_config_t (swiglu_limit and swiglu_alpha are not used;
+ * wfmt must be MOE_W_DENSE, else MOE_ERR_UNSUPPORTED) and the same expert
+ * weight struct, whose bias and scale pointers are ignored.  Ties among the
+ * chosen experts and their order are this library's reading; the page leaves
+ * them to Argpartition.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t norm_topk_prob;               /* nonzero: weights divided by their sum when k > 1 */
+  float routed_scaling_factor;          /* every routing weight is multiplied by it (finite) */
+  const void* e_score_correction_bias;  /* [E] in dtype, added to the scores for the choice only; NULL = none */
+  const void* ws_gate;                  /* shared expert [Fs, D] in dtype (ignored when Fs = 0) */
+  const void* ws_up;                    /* shared expert [Fs, D] */
+  const void* ws_down;                  /* shared expert [D, Fs] */
+  int32_t shared_intermediate_size;     /* Fs: 0 (no shared expert) or a multiple of 16, <= 2^20 */
+} moe_glm_params_t;
+
+/* Bytes of workspace moe_glm_router_topk needs for T tokens (the router's fp32
+ * logits).  (size_t)-1 if cfg is invalid. */
+MOE_API size_t moe_glm_router_workspace_size(const moe_config_t* cfg, int64_t T);
+
+/* Bytes of workspace moe_glm_layer_forward needs for T tokens: as for
+ * moe_layer_forward, plus zero biases for the expert GEMMs and, with a shared
+ * expert, its offsets, SiLU output [T, Fs] and output rows [T, D] in dtype.
+ * (size_t)-1 if cfg or p is invalid. */
+MOE_API size_t moe_glm_workspace_size(const moe_config_t* cfg, const moe_glm_params_t* p, int64_t T);
+
+/* The variant's router: x [T, D], w_router [E, D] in dtype -> topk_ids [T, k]
+ * int32, topk_w [T, k] fp32, as defined above.  ws: moe_glm_router_workspace_size
+ * bytes. */
+MOE_API moe_status_t moe_glm_router_topk(const moe_config_t* cfg, const moe_glm_params_t* p, int64_t T,
+                                         const void* x, const void* w_router, int32_t* topk_ids, float* topk_w,
+                                         void* ws, size_t ws_bytes, void* stream);
+
+/* The whole variant layer: router, dispatch (the same permutation as
+ * moe_permute), SiLU experts, weighted combine plus the shared expert.
+ * x [T, D], y [T, D] in dtype; weights->w_gate, w_up [E, F, D], w_down [E, D, F]
+ * in dtype.  topk_ids_out / topk_w_out optional as in moe_layer_forward.
+ * ws: moe_glm_workspace_size bytes. */
+MOE_API moe_status_t moe_glm_layer_forward(const moe_config_t* cfg, const moe_glm_params_t* p, int64_t T,
+                                           const void* x, const void* w_router, const moe_expert_weights_t* weights,
+                                           void* y, int32_t* topk_ids_out, float* topk_w_out, void* ws,
+                                           size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -41,9 +41,22 @@ class MoeExpertWeights(ctypes.Structure):
         "w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down", "b_gate", "b_up", "b_down")]
 
 
+class MoeGlmParams(ctypes.Structure):
+    _fields_ = [
+        ("norm_topk_prob", ctypes.c_int32),
+        ("routed_scaling_factor", ctypes.c_float),
+        ("e_score_correction_bias", ctypes.c_void_p),
+        ("ws_gate", ctypes.c_void_p),
+        ("ws_up", ctypes.c_void_p),
+        ("ws_down", ctypes.c_void_p),
+        ("shared_intermediate_size", ctypes.c_int32),
+    ]
+
+
 _P = ctypes.c_void_p
 _CFG = ctypes.POINTER(MoeConfig)
 _W = ctypes.POINTER(MoeExpertWeights)
+_GP = ctypes.POINTER(MoeGlmParams)
 _I64 = ctypes.c_int64
 _ST = ctypes.c_int
 
@@ -66,6 +79,10 @@ SIGNATURES = {
     "moe_launch_count": (ctypes.c_uint64, []),
     "moe_set_expert_gemm_variant": (_ST, [ctypes.c_int32]),
     "moe_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "moe_glm_router_workspace_size": (ctypes.c_size_t, [_CFG, _I64]),
+    "moe_glm_workspace_size": (ctypes.c_size_t, [_CFG, _GP, _I64]),
+    "moe_glm_router_topk": (_ST, [_CFG, _GP, _I64, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_glm_layer_forward": (_ST, [_CFG, _GP, _I64, _P, _P, _W, _P, _P, _P, _P, ctypes.c_size_t, _P]),
 }
 
 _lock = threading.Lock()

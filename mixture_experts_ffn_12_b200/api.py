@@ -303,6 +303,128 @@ def layer_forward(cfg: MoeConfig, x: torch.Tensor, w_router: torch.Tensor, b_rou
     return y
 
 
+# --------------------------------------------------------------------------- #
+# the GLM4-MoE-Lite variant (moe_glm_*)
+# --------------------------------------------------------------------------- #
+@dataclasses.dataclass
+class GlmParams:
+    """Router and shared-expert parameters of the GLM4-MoE-Lite variant (moe_glm_params_t):
+    e_score_correction_bias [E] and the shared expert ws_gate / ws_up [Fs, D], ws_down [D, Fs],
+    all in the layer dtype and optional."""
+    norm_topk_prob: bool = True
+    routed_scaling_factor: float = 1.0
+    e_score_correction_bias: Optional[torch.Tensor] = None
+    ws_gate: Optional[torch.Tensor] = None
+    ws_up: Optional[torch.Tensor] = None
+    ws_down: Optional[torch.Tensor] = None
+
+    @property
+    def shared_intermediate_size(self) -> int:
+        return 0 if self.ws_gate is None else int(self.ws_gate.shape[0])
+
+    def c_struct(self) -> _lib.MoeGlmParams:
+        ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        return _lib.MoeGlmParams(1 if self.norm_topk_prob else 0, float(self.routed_scaling_factor),
+                                 ptr(self.e_score_correction_bias), ptr(self.ws_gate), ptr(self.ws_up),
+                                 ptr(self.ws_down), self.shared_intermediate_size)
+
+
+def glm_params_from(spec, d: Dict[str, torch.Tensor]) -> GlmParams:
+    """Parameters of a ``workloads.GlmLayerSpec`` layer uploaded with ``upload_layer``."""
+    return GlmParams(spec.norm_topk_prob, spec.routed_scaling_factor, d.get("e_score_correction_bias"),
+                     d.get("ws_gate"), d.get("ws_up"), d.get("ws_down"))
+
+
+def glm_expert_weights_from(d: Dict[str, torch.Tensor]) -> ExpertWeights:
+    """The variant's expert weights (no biases)."""
+    return ExpertWeights(d["w_gate"], d["w_up"], d["w_down"], None, None, None)
+
+
+def glm_config_from_spec(spec) -> MoeConfig:
+    """Config of a ``workloads.GlmLayerSpec`` (the SwiGLU limit and alpha are not used by the variant)."""
+    return make_config(spec.D, spec.F, spec.E, spec.k, dtype=spec.dtype)
+
+
+def check_glm_args(cfg: MoeConfig, params: GlmParams, x, w_router, weights: Optional[ExpertWeights] = None,
+                   y=None, topk_ids=None, topk_w=None) -> int:
+    """x [T, D], W_r [E, D], e_score_correction_bias [E], the shared expert (all three or none:
+    [Fs, D], [Fs, D], [D, Fs]) and, when given, the expert weights (dense, no biases) and
+    y [T, D], in the layer dtype; topk_ids [T, k] int32 and topk_w [T, k] fp32.  Returns T."""
+    D, F, E, k = cfg.hidden_size, cfg.intermediate_size, cfg.num_local_experts, cfg.num_experts_per_tok
+    dt = torch_dtype(cfg)
+    if cfg.wfmt != _lib.MOE_W_DENSE:
+        raise ValueError("the GLM4-MoE-Lite variant takes dense expert weights")
+    T = _rows("x", x)
+    dev = x.device
+    _want("x", x, (T, D), dt)
+    _want("w_router", w_router, (E, D), dt, dev)
+    if params.e_score_correction_bias is not None:
+        _want("e_score_correction_bias", params.e_score_correction_bias, (E,), dt, dev)
+    shared = [params.ws_gate, params.ws_up, params.ws_down]
+    if any(t is not None for t in shared):
+        Fs = _rows("ws_gate", params.ws_gate)
+        _want("ws_gate", params.ws_gate, (Fs, D), dt, dev)
+        _want("ws_up", params.ws_up, (Fs, D), dt, dev)
+        _want("ws_down", params.ws_down, (D, Fs), dt, dev)
+    if weights is not None:
+        _want("w_gate", weights.w_gate, (E, F, D), dt, dev)
+        _want("w_up", weights.w_up, (E, F, D), dt, dev)
+        _want("w_down", weights.w_down, (E, D, F), dt, dev)
+    if y is not None:
+        _want("y", y, (T, D), dt, dev)
+    if topk_ids is not None:
+        _want("topk_ids", topk_ids, (T, k), torch.int32, dev)
+    if topk_w is not None:
+        _want("topk_w", topk_w, (T, k), torch.float32, dev)
+    return T
+
+
+def glm_router_topk(cfg: MoeConfig, params: GlmParams, x: torch.Tensor, w_router: torch.Tensor,
+                    topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None
+                    ) -> Tuple[torch.Tensor, torch.Tensor]:
+    T = check_glm_args(cfg, params, x, w_router, topk_ids=topk_ids, topk_w=topk_w)
+    L = _lib.load()
+    k, dev = cfg.num_experts_per_tok, x.device
+    if topk_ids is None:
+        topk_ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    nws = _size(L.moe_glm_router_workspace_size(ctypes.byref(cfg), T), "moe_glm_router_workspace_size")
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+    gp = params.c_struct()
+    with torch.cuda.device(dev):
+        _check(L.moe_glm_router_topk(ctypes.byref(cfg), ctypes.byref(gp), T, _p(x), _p(w_router), _p(topk_ids),
+                                     _p(topk_w), _p(ws), ws.numel(), _stream(dev)), "moe_glm_router_topk")
+    return topk_ids, topk_w
+
+
+def glm_workspace_size(cfg: MoeConfig, params: GlmParams, T: int) -> int:
+    gp = params.c_struct()
+    return _size(_lib.load().moe_glm_workspace_size(ctypes.byref(cfg), ctypes.byref(gp), T), "moe_glm_workspace_size")
+
+
+def glm_layer_forward(cfg: MoeConfig, params: GlmParams, x: torch.Tensor, w_router: torch.Tensor,
+                      weights: ExpertWeights, y: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                      topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None
+                      ) -> torch.Tensor:
+    T = check_glm_args(cfg, params, x, w_router, weights, y, topk_ids, topk_w)
+    dev = x.device
+    if y is None:
+        y = torch.empty((T, cfg.hidden_size), dtype=x.dtype, device=dev)
+    if ws is None:
+        ws = torch.empty(max(glm_workspace_size(cfg, params, T), 16), dtype=torch.uint8, device=dev)
+    elif ws.device != dev:
+        raise ValueError(f"ws is on {ws.device}, expected {dev}")
+    wst = weights.c_struct()
+    gp = params.c_struct()
+    with torch.cuda.device(dev):
+        _check(_lib.load().moe_glm_layer_forward(ctypes.byref(cfg), ctypes.byref(gp), T, _p(x), _p(w_router),
+                                                 ctypes.byref(wst), _p(y), _p(topk_ids), _p(topk_w), _p(ws),
+                                                 ws.numel() * ws.element_size(), _stream(dev)),
+               "moe_glm_layer_forward")
+    return y
+
+
 def last_device_error() -> int:
     """Reads and clears the device error word (synchronises); returns a status code."""
     return _lib.load().moe_last_device_error()

@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const float bu = to_f32<T>(static_cast<const T*>(args.bias1)[static_cast<size_t>(ui.g) * args.n_out + f]);
             T* out = static_cast<T*>(args.out);
             for (int c = 0; c < ntok; ++c) {
-              const float gc = fminf(fmaxf(v[c] + bg, 0.0f), args.limit);
+              const float gc = fminf(fmaxf(v[c] + bg, args.gate_lo), args.limit);
               const float uc = fminf(fmaxf(up_stage[wrow * NTOK + c] + bu, -args.limit), args.limit);
               const float h = __fdividef(gc * uc, 1.0f + __expf(-args.alpha * gc));
               out[static_cast<size_t>(ui.m0 + c) * args.ldo + f] = __float2bfloat16_rn(h);

@@ -286,7 +286,7 @@ cudaError_t router_tc(const Launch& L, int64_t T, int D, int E, int k, const voi
 }
 
 // Router with K split over `splits` ranges: tile (m, s) writes fp32 partial logits of
-// tokens m*128.. over K range s to partial[s][T][E]; the top-k kernel sums them.
+// tokens m*128.. over K range s to partial[s][E][T] (expert-major); the top-k kernel sums them.
 cudaError_t router_tc_partial(const Launch& L, int64_t T, int D, int E, int splits, const void* x,
                               const void* w_router, float* partial) {
   const int mma_n = (E + 15) / 16 * 16;
@@ -385,7 +385,8 @@ cudaError_t expert_down_mxfp4(const Launch& L, int64_t R, int D, int F, int E, c
 }
 
 cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,
-                          const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h) {
+                          const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h,
+                          float gate_lo) {
   if (R == 0) return cudaSuccess;
   if (!bf16) {
     GemmArgs a = base_args(L);
@@ -398,6 +399,7 @@ cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, i
     a.bias1 = w.b_up;
     a.limit = limit;
     a.alpha = alpha;
+    a.gate_lo = gate_lo;
     a.out = h;
     a.ldo = F;
     const dim3 grid((F + kSimtBN - 1) / kSimtBN, static_cast<unsigned>((R + kSimtBM - 1) / kSimtBM + E));
@@ -421,6 +423,7 @@ cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, i
   a.bias1 = w.b_up;
   a.limit = limit;
   a.alpha = alpha;
+  a.gate_lo = gate_lo;
   a.out = h;
   a.ldo = F;
   if (gemm_kind(R, E) == GK_DECODE) {
@@ -497,7 +500,9 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
     if ((e = make_tmap(&th, h, false, F, R, 0, kDecTok)) != cudaSuccess) return e;
     const int64_t units = (std::min<int64_t>(E, R) + R / kDecTok) * ((D + 127) / 128);
     if (slot_of_row != nullptr) {
-      if (units <= L.num_sms) {
+      // the split needs a 64-wide K block in each half: with F <= 64 the second half
+      // would be empty and add an accumulator that no MMA wrote
+      if (units <= L.num_sms && (F + 63) / 64 >= 2) {
         // fewer units than SMs (T = 1: 4 experts x 23 feature blocks): split K in two,
         // each half adding its weighted partial into the zeroed fp32 rows
         const int64_t n = R * static_cast<int64_t>(D);

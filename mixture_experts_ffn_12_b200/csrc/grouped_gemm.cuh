@@ -57,6 +57,7 @@ struct GemmArgs {
   const void* bias0;           // [G, n_out] (router: [n_out])
   const void* bias1;           // [G, n_out] (EPI_SWIGLU: up bias)
   float limit, alpha;          // EPI_SWIGLU
+  float gate_lo;               // EPI_SWIGLU: lower clip of the gate (0; -inf with limit = inf, alpha = 1: SiLU(g) * u)
   void* out;                   // output rows
   int ldo;                     // elements between output rows
   const int32_t* slot_of_row;  // EPI_BIAS_WSCATTER
@@ -140,7 +141,7 @@ __device__ __forceinline__ void epi_swiglu(uint32_t tbase, int row, bool rvalid,
       load8<T>(bu + c, b1);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float gc = fminf(fmaxf(g[j] + b0[j], 0.0f), L);
+        const float gc = fminf(fmaxf(g[j] + b0[j], a.gate_lo), L);
         const float uc = fminf(fmaxf(u[j] + b1[j], -L), L);
         h[j] = __fdividef(gc * uc, 1.0f + __expf(-alpha * gc));
       }

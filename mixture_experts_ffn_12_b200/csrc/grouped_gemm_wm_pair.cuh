@@ -103,7 +103,7 @@ __device__ __forceinline__ void wm_epilogue(uint32_t tbase, const WmUnit& un, in
         const float uv = is_up ? v[4 + i] : r;
         const int col = c + (is_up ? 4 + i : i);
         if (fvalid && col < valid) {
-          const float gc = fminf(fmaxf(gv + bg, 0.0f), L);
+          const float gc = fminf(fmaxf(gv + bg, a.gate_lo), L);
           const float uc = fminf(fmaxf(uv + bu, -L), L);
           const float h = __fdividef(gc * uc, 1.0f + __expf(-alpha * gc));
           out[static_cast<size_t>(un.m0 + col) * a.ldo] = __float2bfloat16_rn(h);

@@ -43,8 +43,11 @@ struct ExpertWeights {
 };
 
 // h[R, F] = swiglu(x_perm W_g^T + b_g, x_perm W_u^T + b_u), per expert segment.
+// gate_lo is the gate's lower clip: 0 for the clipped SwiGLU; -inf with limit = inf and
+// alpha = 1 gives SiLU(g) * u.
 cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,
-                          const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h);
+                          const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h,
+                          float gate_lo = 0.0f);
 
 // Down projection.  If slot_of_row == nullptr: out[r] = h[r] W_d^T + b_d (permuted order, dtype);
 // else out[slot_of_row[r]] = topk_w[slot] * (h[r] W_d^T + b_d) (slot order, fp32).

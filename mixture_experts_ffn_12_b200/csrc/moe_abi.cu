@@ -10,6 +10,7 @@
 // one translation unit: the kernels share the per-device error word
 #include "router_permute_combine.cuh"
 #include "gemm_launch.cuh"
+#include "glm_variant.cuh"
 
 namespace {
 
@@ -205,6 +206,58 @@ int32_t* permute_scratch_address(int dev) {
     addr[dev] = static_cast<int32_t*>(p);
   }
   return addr[dev];
+}
+
+// ---------------------------------------------------------------------------
+// the GLM4-MoE-Lite variant
+// ---------------------------------------------------------------------------
+moe_status_t check_glm(const moe_config_t* c, const moe_glm_params_t* p) {
+  moe_status_t s = check_cfg(c);
+  if (s != MOE_OK) return s;
+  if (p == nullptr || !std::isfinite(p->routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
+  const int Fs = p->shared_intermediate_size;
+  if (Fs < 0 || Fs > (1 << 20) || Fs % 16 != 0) return MOE_ERR_INVALID_ARG;
+  if (c->wfmt != MOE_W_DENSE) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+struct GlmLayout {
+  size_t ids, w, off, ros, sor, pscr, xperm, ys, h, rpart, zb, soff, hs, ysh, total;
+};
+
+GlmLayout glm_layout(const moe_config_t* c, const moe_glm_params_t* p, int64_t T) {
+  const size_t R = size_t(T) * c->num_experts_per_tok, es = elem_size(c);
+  const size_t D = c->hidden_size, F = c->intermediate_size, E = c->num_local_experts;
+  const size_t Fs = p->shared_intermediate_size;
+  GlmLayout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.ids = take(R * 4);
+  L.w = take(R * 4);
+  L.off = take((E + 1) * 4);
+  L.ros = take(R * 4);
+  L.sor = take(R * 4);
+  L.pscr = take(moe::permute_scratch_words(T, c->num_local_experts) * 4);
+  L.xperm = take(R * D * (es > 4 ? es : 4));   // x_perm, then the weighted fp32 rows
+  L.ys = L.xperm;
+  const size_t h_bytes = R * F * es, rpart_bytes = moe::router_partial_bytes(T, c->num_local_experts);
+  L.h = take(h_bytes > rpart_bytes ? h_bytes : rpart_bytes);
+  L.rpart = L.h;
+  // zero biases: [E, F] for gate/up, [E, D] for down, [1, Fs] / [1, D] for the shared expert
+  size_t zb = E * (F > D ? F : D);
+  if (Fs > zb) zb = Fs;
+  L.zb = take(zb * es);
+  if (Fs > 0) {
+    L.soff = take(2 * 4);
+    L.hs = take(size_t(T) * Fs * es);
+    L.ysh = take(size_t(T) * D * es);
+  }
+  L.total = o;
+  return L;
 }
 
 }  // namespace
@@ -403,5 +456,113 @@ moe_status_t moe_set_expert_gemm_variant(int32_t variant) {
 }
 
 void moe_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns == 0 ? 1000000000ull : ns); }
+
+size_t moe_glm_router_workspace_size(const moe_config_t* cfg, int64_t T) {
+  if (check_cfg(cfg) != MOE_OK || !check_T(T, cfg->num_experts_per_tok)) return size_t(-1);
+  return moe::router_partial_bytes(T, cfg->num_local_experts);
+}
+
+size_t moe_glm_workspace_size(const moe_config_t* cfg, const moe_glm_params_t* p, int64_t T) {
+  if (check_glm(cfg, p) != MOE_OK || !check_T(T, cfg->num_experts_per_tok)) return size_t(-1);
+  return glm_layout(cfg, p, T).total;
+}
+
+moe_status_t moe_glm_router_topk(const moe_config_t* cfg, const moe_glm_params_t* p, int64_t T, const void* x,
+                                 const void* w_router, int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  moe_status_t s = check_glm(cfg, p);
+  if (s != MOE_OK) return s;
+  if (!check_T(T, cfg->num_experts_per_tok)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!ptr_ok(x) || !ptr_ok(w_router) || !ptr_ok(topk_ids) || !ptr_ok(topk_w)) return MOE_ERR_INVALID_ARG;
+  if (p->e_score_correction_bias != nullptr && !aligned16(p->e_score_correction_bias)) return MOE_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < moe::router_partial_bytes(T, cfg->num_local_experts))
+    return MOE_ERR_WORKSPACE;
+  Launch L;
+  if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
+  return cuda_status(moe::glm_router(L, cfg->dtype == MOE_BF16, T, cfg->hidden_size, cfg->num_local_experts,
+                                     cfg->num_experts_per_tok, x, w_router, p->e_score_correction_bias,
+                                     p->norm_topk_prob != 0, p->routed_scaling_factor, topk_ids, topk_w,
+                                     static_cast<float*>(ws)));
+}
+
+moe_status_t moe_glm_layer_forward(const moe_config_t* cfg, const moe_glm_params_t* p, int64_t T, const void* x,
+                                   const void* w_router, const moe_expert_weights_t* weights, void* y,
+                                   int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  moe_status_t s = check_glm(cfg, p);
+  if (s != MOE_OK) return s;
+  if (!check_T(T, cfg->num_experts_per_tok)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  const int Fs = p->shared_intermediate_size;
+  if (!ptr_ok(x) || !ptr_ok(w_router) || !ptr_ok(y) || weights == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!ptr_ok(weights->w_gate) || !ptr_ok(weights->w_up) || !ptr_ok(weights->w_down)) return MOE_ERR_INVALID_ARG;
+  if (Fs > 0 && (!ptr_ok(p->ws_gate) || !ptr_ok(p->ws_up) || !ptr_ok(p->ws_down))) return MOE_ERR_INVALID_ARG;
+  if (p->e_score_correction_bias != nullptr && !aligned16(p->e_score_correction_bias)) return MOE_ERR_INVALID_ARG;
+  if ((topk_ids_out != nullptr && !aligned16(topk_ids_out)) || (topk_w_out != nullptr && !aligned16(topk_w_out)))
+    return MOE_ERR_INVALID_ARG;
+  const GlmLayout LY = glm_layout(cfg, p, T);
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < LY.total) return MOE_ERR_WORKSPACE;
+  Launch L;
+  if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
+
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t*>(base + LY.ids);
+  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(base + LY.w);
+  int32_t* eoff = reinterpret_cast<int32_t*>(base + LY.off);
+  int32_t* ros = reinterpret_cast<int32_t*>(base + LY.ros);
+  int32_t* sor = reinterpret_cast<int32_t*>(base + LY.sor);
+  int32_t* pscr = reinterpret_cast<int32_t*>(base + LY.pscr);
+  void* xperm = base + LY.xperm;
+  void* h = base + LY.h;
+  void* ys = base + LY.ys;
+  void* zb = base + LY.zb;
+  const bool bf16 = cfg->dtype == MOE_BF16;
+  const int D = cfg->hidden_size, F = cfg->intermediate_size, E = cfg->num_local_experts,
+            k = cfg->num_experts_per_tok;
+  const int64_t R = T * k;
+  const size_t es = elem_size(cfg);
+  // SiLU(g) * u is the clipped SwiGLU with the gate floor at -inf, no upper clip and alpha = 1
+  const float kInf = INFINITY;
+
+  // zero biases for the expert GEMMs (the page's experts have none)
+  size_t zb_elems = size_t(E) * (F > D ? F : D);
+  if (size_t(Fs) > zb_elems) zb_elems = Fs;
+  if (cudaMemsetAsync(zb, 0, zb_elems * es, L.stream) != cudaSuccess) return MOE_ERR_CUDA;
+
+  if (moe::glm_router(L, bf16, T, D, E, k, x, w_router, p->e_score_correction_bias, p->norm_topk_prob != 0,
+                      p->routed_scaling_factor, ids, w, reinterpret_cast<float*>(base + LY.rpart)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (moe::permute(L, bf16, T, D, E, k, ids, x, eoff, ros, sor, xperm, pscr) != cudaSuccess) return MOE_ERR_CUDA;
+  moe::ExpertWeights rw{};
+  rw.w_gate = weights->w_gate;
+  rw.w_up = weights->w_up;
+  rw.w_down = weights->w_down;
+  rw.b_gate = zb;
+  rw.b_up = zb;
+  rw.b_down = zb;
+  if (moe::expert_gateup(L, bf16, R, D, F, E, xperm, eoff, rw, kInf, 1.0f, h, -kInf) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (moe::expert_down(L, bf16, R, D, F, E, h, eoff, rw, sor, w, ys) != cudaSuccess) return MOE_ERR_CUDA;
+  void* ysh = nullptr;
+  if (Fs > 0) {
+    int32_t* soff = reinterpret_cast<int32_t*>(base + LY.soff);
+    void* hs = base + LY.hs;
+    ysh = base + LY.ysh;
+    moe::ExpertWeights sw{};
+    sw.w_gate = p->ws_gate;
+    sw.w_up = p->ws_up;
+    sw.w_down = p->ws_down;
+    sw.b_gate = zb;
+    sw.b_up = zb;
+    sw.b_down = zb;
+    if (moe::glm_shared_off(L, T, soff) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe::expert_gateup(L, bf16, T, D, Fs, 1, x, soff, sw, kInf, 1.0f, hs, -kInf) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (moe::expert_down(L, bf16, T, D, Fs, 1, hs, soff, sw, nullptr, nullptr, ysh) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  return cuda_status(moe::combine_slots_shared(L, bf16, T, D, k, ys, ysh, y));
+}
 
 }  // extern "C"

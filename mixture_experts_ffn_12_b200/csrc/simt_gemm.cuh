@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(256)
       if (n >= N) continue;
       float v;
       if constexpr (EPI == EPI_SWIGLU) {
-        const float gc = fminf(fmaxf(acc0[i][j] + bias0[n], 0.0f), args.limit);
+        const float gc = fminf(fmaxf(acc0[i][j] + bias0[n], args.gate_lo), args.limit);
         const float uc = fminf(fmaxf(acc1[i][j] + bias1[n], -args.limit), args.limit);
         v = gc * uc / (1.0f + expf(-args.alpha * gc));
       } else if constexpr (EPI == EPI_BIAS_WSCATTER) {

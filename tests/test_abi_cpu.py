@@ -34,6 +34,10 @@ def test_every_declared_symbol_is_exported(lib):
 def test_struct_layout_matches_header():
     assert ctypes.sizeof(_lib.MoeConfig) == 32
     assert ctypes.sizeof(_lib.MoeExpertWeights) == 9 * ctypes.sizeof(ctypes.c_void_p)
+    # int32, float, four pointers, int32 (+ tail padding to pointer alignment)
+    assert ctypes.sizeof(_lib.MoeGlmParams) == 48
+    assert _lib.MoeGlmParams.e_score_correction_bias.offset == 8
+    assert _lib.MoeGlmParams.shared_intermediate_size.offset == 40
 
 
 def cfg(**kw):
@@ -129,3 +133,67 @@ def test_rejections_launch_nothing(lib):
         _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_layer_forward(ctypes.byref(c), 0, None, None, None, None, None, None, None, None, 0, None) == \
         _lib.MOE_OK
+
+
+def glm_params(**kw):
+    base = dict(norm_topk_prob=1, routed_scaling_factor=2.5, e_score_correction_bias=None, ws_gate=None,
+                ws_up=None, ws_down=None, shared_intermediate_size=0)
+    base.update(kw)
+    return _lib.MoeGlmParams(**base)
+
+
+def test_glm_workspace_sizes(lib):
+    c = cfg()
+    T, k, D, F, E = 4096, 4, 2880, 2880, 32
+    R = T * k
+    assert lib.moe_glm_router_workspace_size(ctypes.byref(c), T) == 4 * T * E * 4
+    base = lib.moe_glm_workspace_size(ctypes.byref(c), ctypes.byref(glm_params()), T)
+    # as the GPT-OSS layer (maps, x_perm / fp32 rows, h) plus E * max(F, D) zero biases
+    assert base >= R * D * 4 + R * F * 2 + 4 * R * 4 + E * F * 2
+    assert base < R * D * 4 + R * F * 2 + 4 * R * 4 + E * F * 2 + 64 * 1024 * 1024
+    p = ctypes.c_void_p(0x10000).value
+    shared = glm_params(ws_gate=p, ws_up=p, ws_down=p, shared_intermediate_size=1408)
+    # a shared expert adds its offsets, [T, Fs] and [T, D] in bf16
+    extra = lib.moe_glm_workspace_size(ctypes.byref(c), ctypes.byref(shared), T) - base
+    assert T * 1408 * 2 + T * D * 2 <= extra <= T * 1408 * 2 + T * D * 2 + 4 * 256
+    assert lib.moe_glm_workspace_size(ctypes.byref(c), None, T) == _lib.SIZE_INVALID
+    assert lib.moe_glm_workspace_size(ctypes.byref(c), ctypes.byref(glm_params(shared_intermediate_size=24)), T) \
+        == _lib.SIZE_INVALID
+    assert lib.moe_glm_workspace_size(ctypes.byref(cfg(wfmt=_lib.MOE_W_MXFP4)), ctypes.byref(glm_params()), T) \
+        == _lib.SIZE_INVALID
+
+
+def test_glm_rejections_launch_nothing(lib):
+    """The variant's calls return before any CUDA call on bad arguments (no GPU here)."""
+    c = cfg()
+    gp = glm_params()
+    p = ctypes.c_void_p(0x10000)
+    bad = ctypes.c_void_p(0x10008)
+    w = _lib.MoeExpertWeights(*([0x10000] * 3 + [None] * 6))       # the variant's experts have no biases
+    big = 1 << 40
+    fwd = lib.moe_glm_layer_forward
+    assert fwd(ctypes.byref(c), ctypes.byref(gp), 0, None, None, None, None, None, None, None, 0, None) == _lib.MOE_OK
+    assert fwd(ctypes.byref(c), None, 8, p, p, ctypes.byref(w), p, None, None, p, big, None) == \
+        _lib.MOE_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(cfg(wfmt=_lib.MOE_W_MXFP4)), ctypes.byref(gp), 8, p, p, ctypes.byref(w), p, None, None,
+               p, big, None) == _lib.MOE_ERR_UNSUPPORTED
+    assert fwd(ctypes.byref(c), ctypes.byref(glm_params(routed_scaling_factor=float("nan"))), 8, p, p,
+               ctypes.byref(w), p, None, None, p, big, None) == _lib.MOE_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(c), ctypes.byref(gp), 8, bad, p, ctypes.byref(w), p, None, None, p, big, None) == \
+        _lib.MOE_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(c), ctypes.byref(gp), 8, p, p, None, p, None, None, p, big, None) == \
+        _lib.MOE_ERR_INVALID_ARG
+    # a shared expert needs its three matrices
+    sh = glm_params(ws_gate=0x10000, ws_up=None, ws_down=0x10000, shared_intermediate_size=64)
+    assert fwd(ctypes.byref(c), ctypes.byref(sh), 8, p, p, ctypes.byref(w), p, None, None, p, big, None) == \
+        _lib.MOE_ERR_INVALID_ARG
+    # misaligned correction bias
+    cb = glm_params(e_score_correction_bias=0x10004)
+    assert fwd(ctypes.byref(c), ctypes.byref(cb), 8, p, p, ctypes.byref(w), p, None, None, p, big, None) == \
+        _lib.MOE_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(c), ctypes.byref(gp), 8, p, p, ctypes.byref(w), p, None, None, p, 10, None) == \
+        _lib.MOE_ERR_WORKSPACE
+    rt = lib.moe_glm_router_topk
+    assert rt(ctypes.byref(c), ctypes.byref(gp), 0, None, None, None, None, None, 0, None) == _lib.MOE_OK
+    assert rt(ctypes.byref(c), ctypes.byref(gp), 8, p, p, p, p, p, 16, None) == _lib.MOE_ERR_WORKSPACE
+    assert rt(ctypes.byref(c), ctypes.byref(gp), 8, p, None, p, p, p, big, None) == _lib.MOE_ERR_INVALID_ARG

@@ -116,3 +116,37 @@ def test_mxfp4_weights_need_codes_and_scales():
     _expect_refused(api.check_expert_weights, cfg,
                     dataclasses.replace(ew, s_up=torch.empty((E, F, D // 16), dtype=torch.uint8)),
                     match="s_up: shape")
+
+
+GLM_SPECS = [W.glm_tiny_spec(T=7, D=16, E=6, k=2, F=16, F_shared=32, dtype="f32"),
+             W.glm_tiny_spec(T=5, D=32, E=4, k=3, F=16, F_shared=0, dtype="bf16", correction_b_std=None, cfg_id=311)]
+
+
+@pytest.mark.parametrize("spec", GLM_SPECS, ids=lambda s: s.name)
+def test_glm_arrays_pass_the_variant_checks(spec):
+    d = {k: api.to_torch(v) for k, v in W.make_glm_layer(spec).items()}
+    cfg = api.glm_config_from_spec(spec)
+    params = api.glm_params_from(spec, d)
+    assert params.shared_intermediate_size == spec.F_shared
+    T, k = spec.T, spec.k
+    assert api.check_glm_args(cfg, params, d["x"], d["w_router"], api.glm_expert_weights_from(d),
+                              torch.empty_like(d["x"]), torch.empty((T, k), dtype=torch.int32),
+                              torch.empty((T, k))) == T
+    c = params.c_struct()
+    assert c.shared_intermediate_size == spec.F_shared and c.norm_topk_prob == int(spec.norm_topk_prob)
+
+
+def test_glm_mismatches_are_refused():
+    spec = GLM_SPECS[0]
+    d = {k: api.to_torch(v) for k, v in W.make_glm_layer(spec).items()}
+    cfg = api.glm_config_from_spec(spec)
+    params = api.glm_params_from(spec, d)
+    x, wr = d["x"], d["w_router"]
+    _expect_refused(api.check_glm_args, cfg, dataclasses.replace(params, ws_up=None), x, wr, match="ws_up is required")
+    _expect_refused(api.check_glm_args, cfg,
+                    dataclasses.replace(params, ws_down=params.ws_down.t().contiguous()), x, wr, match="ws_down: shape")
+    _expect_refused(api.check_glm_args, cfg,
+                    dataclasses.replace(params, e_score_correction_bias=torch.zeros(spec.E + 1)), x, wr,
+                    match="e_score_correction_bias: shape")
+    mx = api.make_config(spec.D, spec.F, spec.E, spec.k, dtype="bf16", wfmt="mxfp4")
+    _expect_refused(api.check_glm_args, mx, params, x, wr, match="dense expert weights")

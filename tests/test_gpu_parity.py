@@ -39,7 +39,12 @@ MXFP4_SMALL = W.tiny_spec(T=280, D=128, E=6, k=2, F=160, dtype="bf16", wfmt="mxf
 PAIR_RAGGED = W.tiny_spec(T=900, D=256, E=5, k=2, F=272, dtype="bf16", cfg_id=206, dead_experts=(3,),
                           router_w_std=0.2)
 
-SMALL_SPECS = [W.TINY_FP32, RAGGED_BF16, RAGGED_F32, WIDE_K, ONE_EXPERT, MXFP4_SMALL, PAIR_RAGGED]
+# <= 16 rows per expert with F = 64: the decode kernels by default, with fewer down units than
+# SMs but a single 64-wide K block, so the down projection must not split K (an empty half
+# would add an accumulator no MMA wrote)
+DECODE_ONE_KBLOCK = W.tiny_spec(T=24, D=64, E=16, k=4, F=64, dtype="bf16", cfg_id=210, router_w_std=0.2)
+
+SMALL_SPECS = [W.TINY_FP32, RAGGED_BF16, RAGGED_F32, WIDE_K, ONE_EXPERT, MXFP4_SMALL, PAIR_RAGGED, DECODE_ONE_KBLOCK]
 
 # many experts: the K-split router with 16 / 32 threads per token in its top-k (E = 128 / 256),
 # 256 expert groups in the GEMMs (the maximum), k = 8 (the maximum)

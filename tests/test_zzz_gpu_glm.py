@@ -1,0 +1,121 @@
+"""The GLM4-MoE-Lite variant on the GPU against its CPU oracle, through the C ABI (marked gpu).
+
+Source of the variant: "Ollama glm4_moe_lite.go" (MoEGate.Forward, SwitchMLP.Forward,
+SharedExperts.Forward, MoE.Forward).  Bit-exact: the chosen expert sets (and their
+order where the corrected scores are separated).  Routing weights within 2e-5 (they
+include routed_scaling_factor).  Layer output within 2e-2 of the output's RMS plus
+its own storage rounding, the bound of the GPT-OSS layer.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import glm_moe as G
+from parity_util import TOL_W, TOL_Y, check_ids, check_output, f64
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def api(cuda_ok):
+    from mixture_experts_ffn_12_b200 import api as A, build
+    build.build()
+    return A
+
+
+# T >= 256 with D = 256 (bf16): the tensor-core router with its K split; fewer tokens
+# or fp32: the SIMT router.  <= 16 rows per expert on average: the decode kernels.
+GLM_TC_ROUTER = W.glm_tiny_spec(T=300, D=256, E=8, k=2, F=144, F_shared=96, dtype="bf16", cfg_id=330)
+GLM_F32 = W.glm_tiny_spec(T=77, D=96, E=5, k=3, F=48, F_shared=32, dtype="f32", cfg_id=331)
+GLM_DECODE = W.glm_tiny_spec(T=40, D=64, E=16, k=4, F=64, F_shared=0, dtype="bf16", norm_topk_prob=False,
+                             routed_scaling_factor=1.0, correction_b_std=None, cfg_id=332)
+GLM_K1 = W.glm_tiny_spec(T=20, D=32, E=4, k=1, F=32, F_shared=32, dtype="bf16", cfg_id=333)
+GLM_KE = W.glm_tiny_spec(T=30, D=32, E=4, k=4, F=32, F_shared=16, dtype="bf16", cfg_id=334)
+GLM_MANY = W.glm_tiny_spec(T=300, D=256, E=64, k=6, F=64, F_shared=64, dtype="bf16", router_w_std=0.1, cfg_id=335)
+SPECS = [GLM_TC_ROUTER, GLM_F32, GLM_DECODE, GLM_K1, GLM_KE, GLM_MANY]
+
+
+def _scores_fn(spec):
+    def f(layer):
+        return G.route(G.gate_logits(layer["x"], layer["w_router"]), spec.k, layer.get("e_score_correction_bias"))[3]
+    return f
+
+
+def _layer(spec):
+    return W.make_glm_layer(spec, seed=0, scores_fn=_scores_fn(spec))
+
+
+def _run(api, spec, layer):
+    d = api.upload_layer(layer)
+    cfg = api.glm_config_from_spec(spec)
+    params = api.glm_params_from(spec, d)
+    ids = torch.empty((spec.T, spec.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((spec.T, spec.k), dtype=torch.float32, device="cuda")
+    y = api.glm_layer_forward(cfg, params, d["x"], d["w_router"], api.glm_expert_weights_from(d),
+                              topk_ids=ids, topk_w=w)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    return y, ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+
+
+def _check_weights(gid, gw, rid, rw):
+    got = np.take_along_axis(gw, np.argsort(gid, axis=1), axis=1)
+    ref = np.take_along_axis(rw, np.argsort(rid, axis=1), axis=1)
+    assert np.max(np.abs(got - ref)) <= TOL_W
+
+
+@pytest.mark.parametrize("spec", SPECS, ids=lambda s: s.name)
+def test_glm_layer_forward(api, spec):
+    layer = _layer(spec)
+    y, gid, gw = _run(api, spec, layer)
+    ref = G.layer_forward(layer, spec.k, spec.norm_topk_prob, spec.routed_scaling_factor)
+    check_ids(gid, ref["ids"], ref["chosen_by"])
+    _check_weights(gid, gw, ref["ids"], ref["w"])
+    check_output(f64(y), ref["y"], TOL_Y[spec.dtype], spec.dtype == "bf16")
+
+
+@pytest.mark.parametrize("spec", [GLM_TC_ROUTER, GLM_F32, GLM_K1, GLM_MANY], ids=lambda s: s.name)
+def test_glm_router_topk(api, spec):
+    layer = _layer(spec)
+    d = api.upload_layer({k: layer[k] for k in layer if k in ("x", "w_router", "e_score_correction_bias")})
+    ids, w = api.glm_router_topk(api.glm_config_from_spec(spec), api.glm_params_from(spec, d), d["x"], d["w_router"])
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    rid, rw, _, chosen_by = G.route(G.gate_logits(layer["x"], layer["w_router"]), spec.k,
+                                    layer.get("e_score_correction_bias"), spec.norm_topk_prob,
+                                    spec.routed_scaling_factor)
+    gid = ids.cpu().numpy()
+    check_ids(gid, rid, chosen_by)
+    _check_weights(gid, w.cpu().numpy().astype(np.float64), rid, rw)
+    if spec.k > 1 and spec.norm_topk_prob:
+        np.testing.assert_allclose(w.sum(dim=1).cpu().numpy(), spec.routed_scaling_factor, rtol=1e-6)
+
+
+@pytest.mark.parametrize("variant", [1, 2, 3, 4], ids=["single_cta", "cta_pair", "decode", "wm_pair"])
+def test_glm_each_gemm_variant(api, variant):
+    """SiLU(g) * u through every bf16 expert-GEMM kernel (routed and shared experts)."""
+    spec = GLM_TC_ROUTER
+    layer = _layer(spec)
+    api.set_expert_gemm_variant(variant)
+    try:
+        y, gid, _ = _run(api, spec, layer)
+    finally:
+        api.set_expert_gemm_variant(0)
+    ref = G.layer_forward(layer, spec.k, spec.norm_topk_prob, spec.routed_scaling_factor)
+    check_ids(gid, ref["ids"], ref["chosen_by"])
+    check_output(f64(y), ref["y"], TOL_Y["bf16"], True)
+
+
+def test_glm_zero_tokens(api):
+    from mixture_experts_ffn_12_b200 import _lib
+    spec = W.glm_tiny_spec(T=0, D=32, E=4, k=2, F=32, F_shared=16, dtype="bf16", cfg_id=336)
+    d = api.upload_layer(W.make_glm_layer(spec))
+    lib = _lib.load()
+    before = lib.moe_launch_count()
+    y = api.glm_layer_forward(api.glm_config_from_spec(spec), api.glm_params_from(spec, d), d["x"], d["w_router"],
+                              api.glm_expert_weights_from(d))
+    torch.cuda.synchronize()
+    assert tuple(y.shape) == (0, spec.D)
+    assert lib.moe_launch_count() == before
