@@ -50,6 +50,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-decode", action="store_true", help="skip the decode-regime sweep")
     p.add_argument("--no-mxfp4", action="store_true", help="skip the MXFP4-weight layer")
+    p.add_argument("--no-skewed", action="store_true", help="skip the GPT-OSS-120B-shaped skewed layer")
+    p.add_argument("--no-glm", action="store_true", help="skip the GLM4-MoE-Lite variant layer")
     return p.parse_args()
 
 
@@ -305,11 +307,17 @@ def run_ours(args, rank, world, local_rank):
     ms_e2e = max_over_ranks(e0.elapsed_time(e1))
 
     decode = decode_sweep(api, moe, spec, layer, dev, stream, max(20, K // 4)) if not args.no_decode else None
-    mx = None
-    if not args.no_mxfp4 and world == 1 and spec.wfmt == "dense" and spec.dtype == "bf16":
+    mx = sk = glm = None
+    extra = world == 1 and spec.name == W.GPTOSS20B_PREFILL.name
+    if extra:
         del d, moe
         torch.cuda.empty_cache()
-        mx = mxfp4_sweep(api, dev, stream, max(10, K // 10))
+        if not args.no_mxfp4:
+            mx = mxfp4_sweep(api, dev, stream, max(10, K // 10))
+        if not args.no_skewed:
+            sk = skewed_sweep(api, dev, stream, max(10, K // 2))
+        if not args.no_glm:
+            glm = glm_sweep(api, dev, stream, max(10, K // 2))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -348,6 +356,10 @@ def run_ours(args, rank, world, local_rank):
             line["decode"] = decode
         if mx is not None:
             line["mxfp4"] = mx
+        if sk is not None:
+            line["skewed"] = sk
+        if glm is not None:
+            line["glm_variant"] = glm
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
@@ -355,41 +367,192 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
-def decode_sweep(api, moe, spec, layer, dev, stream, steps):
+def decode_sweep(api, moe, spec, layer, dev, stream, steps, copies=4):
     """Decode regime of the same layer (T = 1, 8, 32, 64): GB/s of the expert weights the step touches.
 
     Each step replays a CUDA graph of one moe_layer_forward (same kernels, no host launch overhead).
+    The replays rotate over `copies` copies of the expert weights (each its own MoELayer and graph),
+    so a step's weights were last read `copies` - 1 steps earlier, at least 4 x 199 MB (T = 1) of
+    other weights ago: more than L2 holds, so every step streams its weights from HBM.
     Touched bytes = (experts with at least one routed token) x 3 x D x F x element size, plus the
-    router weights; each step streams them from HBM (T = 1 touches 4 experts = 0.2 GB > L2).
+    router weights.
     """
     import torch
     peaks = measured_peaks()
-    out = {}
+    out = {"weight_copies": copies}
     esz = 2 if spec.dtype == "bf16" else 4
+    ew = moe.experts
+    layers = [moe]
+    for _ in range(copies - 1):
+        cp = api.ExpertWeights(*(None if t is None else t.clone() for t in
+                                 (ew.w_gate, ew.w_up, ew.w_down, ew.b_gate, ew.b_up, ew.b_down)),
+                               *(None if t is None else t.clone() for t in (ew.s_gate, ew.s_up, ew.s_down)))
+        layers.append(api.MoELayer(moe.cfg, moe.w_router, moe.b_router, cp))
     for T in W.GPTOSS20B_DECODE_T:
         dspec = W.gptoss20b_decode(T) if spec.name.startswith("gptoss20b") else spec.with_tokens(T)
         x = api.to_torch(W.make_layer(dspec, seed=0, with_experts=False)["x"]).to(dev)
-        y = torch.empty_like(x)
         ids = torch.empty((T, spec.k), dtype=torch.int32, device=dev)
         for _ in range(5):
-            moe(x, y=y, topk_ids=ids)
+            moe(x, topk_ids=ids)
         torch.cuda.synchronize()
         touched = int(torch.unique(ids).numel())
-        # CUDA-graph replay of the same launches (host launch overhead removed)
-        replay, _ = moe.graphed(x, y=y, topk_ids=ids)
-        for _ in range(3):
-            replay()
+        # CUDA-graph replay of the same launches (host launch overhead removed), one graph per copy
+        replays = [lyr.graphed(x, topk_ids=torch.empty_like(ids))[0] for lyr in layers]
+        for i in range(3 * copies):
+            replays[i % copies]()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(steps, 2 * copies)
         a.record(stream)
-        for _ in range(steps):
-            replay()
+        for i in range(n):
+            replays[i % copies]()
         b.record(stream)
         torch.cuda.synchronize()
-        us = 1e3 * a.elapsed_time(b) / steps
+        us = 1e3 * a.elapsed_time(b) / n
         nbytes = touched * 3 * spec.D * spec.F * esz + spec.E * spec.D * esz
         gbs = nbytes / (us * 1e-6) / 1e9
         out[f"T{T}"] = {"us_per_step": us, "experts_touched": touched, "weight_bytes": nbytes, "GB/s": gbs,
                         "hbm_frac": gbs / peaks["hbm_gbs"], "tokens/s": T / (us * 1e-6)}
+        del replays
+    del layers
+    torch.cuda.empty_cache()
+    return out
+
+
+def device_experts(api, spec, dev, seed=0):
+    """Dense bf16 expert weights drawn on the device (torch's generator, seeded), with the
+    recipe's value laws: W ~ N(0, 1/sqrt(fan_in)), biases N(0, expert_b_std).  Timing only:
+    the values do not change the work, and drawing 6.4 GB on the host would take a minute."""
+    import math
+    import torch
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000003 * (seed + 1) + spec.cfg_id)
+    E, D, F = spec.E, spec.D, spec.F
+
+    def w(n, kdim):
+        t = torch.empty((E, n, kdim), dtype=torch.bfloat16, device=dev)
+        for e in range(E):
+            t[e] = (torch.randn((n, kdim), generator=g, device=dev) / math.sqrt(kdim)).to(torch.bfloat16)
+        return t
+
+    def b(n):
+        return (torch.randn((E, n), generator=g, device=dev) * spec.expert_b_std).to(torch.bfloat16)
+
+    return api.ExpertWeights(w(F, D), w(F, D), w(D, F), b(F), b(F), b(D))
+
+
+def timed_steps(fn, stream, steps):
+    """Mean ms per call of fn over `steps` back-to-back calls, CUDA events on `stream`."""
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def stage_times(fn, stream, steps):
+    """Mean ms of each library stage over `steps` calls (separate pass: stage events between kernels)."""
+    import torch
+    from mixture_experts_ffn_12_b200 import _lib
+    lib = _lib.load()
+    n = len(STAGES)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        hs = [ctypes_ptr(e.cuda_event) for e in ev[i]]
+        lib.moe_set_stage_events((_lib.ctypes.c_void_p * n)(*hs[:n]), (_lib.ctypes.c_void_p * n)(*hs[n:]), n)
+        fn()
+    lib.moe_set_stage_events(None, None, 0)
+    torch.cuda.synchronize()
+    return {name: statistics.mean(ev[i][j].elapsed_time(ev[i][n + j]) for i in range(steps))
+            for j, name in enumerate(STAGES)}
+
+
+def skewed_sweep(api, dev, stream, steps):
+    """The GPT-OSS-120B-shaped skewed-load layer (T = 16384, E = 128, k = 4, Zipf(1.1) router
+    bias): step time, tokens/s, TFLOP/s, the touched expert weights and the fraction of the
+    roofline max(FLOP / tensor peak, touched bytes / HBM bandwidth)."""
+    import torch
+    spec = W.GPTOSS120B_SKEWED
+    peaks = measured_peaks()
+    layer = W.make_layer(spec, seed=0, with_experts=False)
+    d = api.upload_layer(layer, dev)
+    moe = api.MoELayer(api.config_from_spec(spec), d["w_router"], d["b_router"], device_experts(api, spec, dev))
+    x = d["x"]
+    y = torch.empty_like(x)
+    ids = torch.empty((spec.T, spec.k), dtype=torch.int32, device=dev)
+    for _ in range(3):
+        moe(x, y=y, topk_ids=ids)
+    torch.cuda.synchronize()
+    if api.last_device_error() != 0:
+        raise RuntimeError("device error word set during the skewed-layer warm-up")
+    cnt = torch.bincount(ids.flatten().long(), minlength=spec.E)
+    touched = int((cnt > 0).sum())
+    ms = timed_steps(lambda: moe(x, y=y), stream, steps)
+    stage = stage_times(lambda: moe(x, y=y), stream, min(steps, 10))
+    if api.last_device_error() != 0:
+        raise RuntimeError("device error word set during the skewed-layer steps")
+    flops = spec.expert_flops() + spec.router_flops()
+    nbytes = touched * 3 * spec.D * spec.F * 2
+    roof_ms = 1e3 * max(flops / (peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+    out = {"workload": spec.name, "T": spec.T, "us_per_step": 1e3 * ms, "tokens/s": spec.T / (ms * 1e-3),
+           "tflops": flops / (ms * 1e-3) / 1e12, "experts_touched": touched,
+           "max_expert_rows": int(cnt.max()), "touched_weight_bytes": nbytes,
+           "roofline_us": 1e3 * roof_ms, "frac": roof_ms / ms,
+           "stage_us": {k: 1e3 * v for k, v in stage.items()},
+           "weights": "expert weights drawn on the device (same law as the recipe); x and router from the recipe"}
+    del moe, d
+    torch.cuda.empty_cache()
+    return out
+
+
+def glm_sweep(api, dev, stream, steps):
+    """The GLM4-MoE-Lite variant at the GPT-OSS-20B shape (T = 4096, E = 32, k = 4, D = F = 2880,
+    a shared expert of 2880): step time, tokens/s and TFLOP/s of the routed and shared experts."""
+    import math
+    import torch
+    spec = W.GLM_GPTOSS20B_SHAPE
+    peaks = measured_peaks()
+    rng = np.random.default_rng(spec.cfg_id)
+    D, E, F, Fs, T = spec.D, spec.E, spec.F, spec.F_shared, spec.T
+    x = api.to_torch(W.f32_to_bf16_bits(rng.standard_normal((T, D), dtype=np.float32))).to(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(spec.cfg_id)
+
+    def mat(*shape, std):
+        return (torch.randn(shape, generator=g, device=dev) * std).to(torch.bfloat16)
+
+    w_router = mat(E, D, std=1 / math.sqrt(D))
+    corr = mat(E, std=spec.correction_b_std)
+    ew = api.ExpertWeights(mat(E, F, D, std=1 / math.sqrt(D)), mat(E, F, D, std=1 / math.sqrt(D)),
+                           mat(E, D, F, std=1 / math.sqrt(F)), None, None, None)
+    params = api.GlmParams(spec.norm_topk_prob, spec.routed_scaling_factor, corr, mat(Fs, D, std=1 / math.sqrt(D)),
+                           mat(Fs, D, std=1 / math.sqrt(D)), mat(D, Fs, std=1 / math.sqrt(Fs)))
+    cfg = api.glm_config_from_spec(spec)
+    y = torch.empty_like(x)
+    ws = torch.empty(api.glm_workspace_size(cfg, params, T), dtype=torch.uint8, device=dev)
+
+    def step():
+        api.glm_layer_forward(cfg, params, x, w_router, ew, y=y, ws=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ms = timed_steps(step, stream, steps)
+    if api.last_device_error() != 0:
+        raise RuntimeError("device error word set during the GLM variant steps")
+    flops = 6.0 * T * spec.k * D * F + 6.0 * T * D * Fs + 2.0 * T * D * E
+    out = {"workload": spec.name, "T": T, "F_shared": Fs, "us_per_step": 1e3 * ms, "tokens/s": T / (ms * 1e-3),
+           "tflops": flops / (ms * 1e-3) / 1e12, "frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+           "weights": "drawn on the device (x from numpy, both seeded)"}
+    del ew, params, ws
+    torch.cuda.empty_cache()
     return out
 
 
@@ -398,7 +561,6 @@ def mxfp4_sweep(api, dev, stream, steps):
     stage times and the gate/up GEMM's TFLOP/s.  The MXFP4 weights are decoded to bf16 inside
     the GEMM mainloop; the FLOPs counted are the bf16 MMA work (4*R*D*F for gate/up)."""
     import torch
-    from mixture_experts_ffn_12_b200 import _lib
     spec = W.GPTOSS20B_MXFP4
     peaks = measured_peaks()
     layer = W.make_layer(spec, seed=0)
@@ -409,27 +571,10 @@ def mxfp4_sweep(api, dev, stream, steps):
     for _ in range(3):
         moe(x, y=y)
     torch.cuda.synchronize()
-    lib = _lib.load()
-    n = len(STAGES)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(steps)]
-    for row in ev:
-        for e in row:
-            e.record(stream)
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for i in range(steps):
-        hs = [ctypes_ptr(e.cuda_event) for e in ev[i]]
-        lib.moe_set_stage_events((_lib.ctypes.c_void_p * n)(*hs[:n]), (_lib.ctypes.c_void_p * n)(*hs[n:]), n)
-        moe(x, y=y)
-    b.record(stream)
-    lib.moe_set_stage_events(None, None, 0)
-    torch.cuda.synchronize()
+    us = 1e3 * timed_steps(lambda: moe(x, y=y), stream, steps)
+    stage = {k: 1e3 * v for k, v in stage_times(lambda: moe(x, y=y), stream, steps).items()}
     if api.last_device_error() != 0:
         raise RuntimeError("device error word set during the MXFP4 steps")
-    us = 1e3 * a.elapsed_time(b) / steps
-    stage = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][n + j]) for i in range(steps)) * 1e3
-             for j, name in enumerate(STAGES)}
     gu_tf = 4.0 * spec.R * spec.D * spec.F / (stage["gateup_swiglu_gemm"] * 1e-6) / 1e12
     return {"workload": spec.name, "T": spec.T, "us_per_step": us, "tokens/s": spec.T / (us * 1e-6),
             "stage_us": stage, "gateup_tflops": gu_tf, "gateup_frac": gu_tf / peaks["bf16_tflops"],

@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -93,6 +93,11 @@ typedef struct {
   float swiglu_alpha;          /* 1.702 for GPT-OSS */
   int32_t dtype;               /* moe_dtype_t */
   int32_t wfmt;                /* moe_wfmt_t */
+  int32_t y_f32;               /* 0: the layer output y is stored in dtype; 1: y is stored in fp32,
+                                  i.e. the fp32 sums before their rounding to dtype (for a bf16
+                                  layer the dtype output is exactly the round-to-nearest-even
+                                  of this fp32 output).  Applies to moe_layer_forward,
+                                  moe_combine and moe_glm_layer_forward. */
 } moe_config_t;
 
 /* Expert parameters (device pointers).  Dense: w_* in dtype, s_* NULL.
@@ -169,9 +174,12 @@ MOE_API moe_status_t moe_permute(const moe_config_t* cfg, int64_t T, const int32
  *    one per GPU that loads the library, held until the process exits), so
  *    num_local_experts * ceil(T / 256) must be at most 32768 (e.g. T <= 65536
  *    with E = 128); larger sizes return MOE_ERR_UNSUPPORTED and launch nothing;
- *  - the first call on a device looks up that array's device address (a
- *    runtime call, no allocation); make that first call before any stream
- *    capture;
+ *  - each call finds that array's device address in the current CUDA context
+ *    (cudaGetSymbolAddress, a runtime call that allocates nothing); the first
+ *    call in a context does the lookup and caches it for that context (keyed by
+ *    its unique context id, so a context of the caller's own or the one made
+ *    after cudaDeviceReset gets a fresh lookup); make that first call before
+ *    any stream capture;
  *  - every call on a device shares the array and it keeps the last call's
  *    contents (each call writes every word it reads, so nothing needs clearing),
  *    hence calls that may overlap on the GPU (other streams, other threads) race
@@ -195,13 +203,16 @@ MOE_API moe_status_t moe_expert_ffn(const moe_config_t* cfg, int64_t T, const vo
                             void* stream);
 
 /* Weighted combine: y[t] = sum_{j<k} topk_w[t,j] * y_perm[row_of_slot[t,j]],
- * summed in fp32 in fixed j order.  y_perm [T*k, D], y [T, D] in dtype. */
+ * summed in fp32 in fixed j order.  y_perm [T*k, D] in dtype; y [T, D] in dtype,
+ * or in fp32 when cfg->y_f32 is set. */
 MOE_API moe_status_t moe_combine(const moe_config_t* cfg, int64_t T, const void* y_perm, const int32_t* row_of_slot,
                          const float* topk_w, void* y, void* stream);
 
 /* The whole layer: router/top-k -> dispatch -> gate/up + SwiGLU -> down with
  * the routing weight and the un-permutation fused into its epilogue -> sum
- * over k.  x [T, D], y [T, D] in dtype.  topk_ids_out [T, k] and topk_w_out
+ * over k.  x [T, D] in dtype; y [T, D] in dtype, or in fp32 when cfg->y_f32
+ * is set (the k weighted expert outputs are summed in fp32 either way; a dtype
+ * output is that sum rounded once).  topk_ids_out [T, k] and topk_w_out
  * [T, k] are optional (NULL: kept in the workspace).  ws: moe_workspace_size
  * bytes. */
 MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x, const void* w_router,
@@ -276,7 +287,8 @@ MOE_API size_t moe_glm_router_workspace_size(const moe_config_t* cfg, int64_t T)
 
 /* Bytes of workspace moe_glm_layer_forward needs for T tokens: as for
  * moe_layer_forward, plus zero biases for the expert GEMMs and, with a shared
- * expert, its offsets, SiLU output [T, Fs] and output rows [T, D] in dtype.
+ * expert, its offsets, identity slot map and unit weights [T], SiLU output
+ * [T, Fs] in dtype and fp32 output rows [T, D].
  * (size_t)-1 if cfg or p is invalid. */
 MOE_API size_t moe_glm_workspace_size(const moe_config_t* cfg, const moe_glm_params_t* p, int64_t T);
 
@@ -289,8 +301,9 @@ MOE_API moe_status_t moe_glm_router_topk(const moe_config_t* cfg, const moe_glm_
 
 /* The whole variant layer: router, dispatch (the same permutation as
  * moe_permute), SiLU experts, weighted combine plus the shared expert.
- * x [T, D], y [T, D] in dtype; weights->w_gate, w_up [E, F, D], w_down [E, D, F]
- * in dtype.  topk_ids_out / topk_w_out optional as in moe_layer_forward.
+ * x [T, D] in dtype; y [T, D] in dtype (fp32 when cfg->y_f32 is set); the
+ * routed and shared expert outputs are summed in fp32 and rounded once.
+ * weights->w_gate, w_up [E, F, D], w_down [E, D, F] in dtype.  topk_ids_out / topk_w_out optional as in moe_layer_forward.
  * ws: moe_glm_workspace_size bytes. */
 MOE_API moe_status_t moe_glm_layer_forward(const moe_config_t* cfg, const moe_glm_params_t* p, int64_t T,
                                            const void* x, const void* w_router, const moe_expert_weights_t* weights,

@@ -21,6 +21,7 @@ MOE_F32, MOE_BF16 = 0, 1
 MOE_W_DENSE, MOE_W_MXFP4 = 0, 1
 
 SIZE_INVALID = ctypes.c_size_t(-1).value
+ABI_VERSION = 2
 
 
 class MoeConfig(ctypes.Structure):
@@ -33,6 +34,7 @@ class MoeConfig(ctypes.Structure):
         ("swiglu_alpha", ctypes.c_float),
         ("dtype", ctypes.c_int32),
         ("wfmt", ctypes.c_int32),
+        ("y_f32", ctypes.c_int32),
     ]
 
 
@@ -102,7 +104,7 @@ def load() -> ctypes.CDLL:
                 fn = getattr(lib, name)
                 fn.restype = res
                 fn.argtypes = args
-            if lib.moe_abi_version() != 1:
+            if lib.moe_abi_version() != ABI_VERSION:
                 raise RuntimeError("libmoe ABI version mismatch")
             _lib = lib
         return _lib

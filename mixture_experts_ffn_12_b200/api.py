@@ -35,18 +35,25 @@ _DT = {"bf16": (_lib.MOE_BF16, torch.bfloat16), "f32": (_lib.MOE_F32, torch.floa
 
 def make_config(hidden_size: int, intermediate_size: int, num_local_experts: int, num_experts_per_tok: int,
                 swiglu_limit: float = 7.0, swiglu_alpha: float = 1.702, dtype: str = "bf16",
-                wfmt: str = "dense") -> MoeConfig:
+                wfmt: str = "dense", y_f32: bool = False) -> MoeConfig:
+    """y_f32: the layer output y is stored in fp32 (the sums before their rounding to dtype)."""
     return MoeConfig(hidden_size, intermediate_size, num_local_experts, num_experts_per_tok, swiglu_limit,
-                     swiglu_alpha, _DT[dtype][0], _lib.MOE_W_MXFP4 if wfmt == "mxfp4" else _lib.MOE_W_DENSE)
+                     swiglu_alpha, _DT[dtype][0], _lib.MOE_W_MXFP4 if wfmt == "mxfp4" else _lib.MOE_W_DENSE,
+                     1 if y_f32 else 0)
 
 
-def config_from_spec(spec) -> MoeConfig:
+def config_from_spec(spec, y_f32: bool = False) -> MoeConfig:
     """Config of a ``workloads.LayerSpec``."""
-    return make_config(spec.D, spec.F, spec.E, spec.k, spec.limit, spec.alpha, spec.dtype, spec.wfmt)
+    return make_config(spec.D, spec.F, spec.E, spec.k, spec.limit, spec.alpha, spec.dtype, spec.wfmt, y_f32)
 
 
 def torch_dtype(cfg: MoeConfig) -> torch.dtype:
     return torch.bfloat16 if cfg.dtype == _lib.MOE_BF16 else torch.float32
+
+
+def out_dtype(cfg: MoeConfig) -> torch.dtype:
+    """dtype of the layer output y: fp32 when cfg.y_f32 is set, else the layer dtype."""
+    return torch.float32 if cfg.y_f32 else torch_dtype(cfg)
 
 
 def _p(t: Optional[torch.Tensor]):
@@ -160,12 +167,12 @@ def check_combine_args(cfg: MoeConfig, y_perm, row_of_slot, topk_w) -> int:
 def check_layer_args(cfg: MoeConfig, x, w_router, b_router, weights: Optional["ExpertWeights"], y=None,
                      topk_ids=None, topk_w=None) -> int:
     """The router's arguments, the expert weights (skipped when None: already checked)
-    and y [T, D] in the layer dtype when given.  Returns T."""
+    and y [T, D] in the output dtype (``out_dtype``) when given.  Returns T."""
     T = check_router_args(cfg, x, w_router, b_router, topk_ids, topk_w)
     if weights is not None:
         check_expert_weights(cfg, weights, x.device)
     if y is not None:
-        _want("y", y, (T, cfg.hidden_size), torch_dtype(cfg), x.device)
+        _want("y", y, (T, cfg.hidden_size), out_dtype(cfg), x.device)
     return T
 
 
@@ -272,7 +279,7 @@ def expert_ffn(cfg: MoeConfig, x_perm: torch.Tensor, expert_off: torch.Tensor, w
 def combine(cfg: MoeConfig, y_perm: torch.Tensor, row_of_slot: torch.Tensor, topk_w: torch.Tensor) -> torch.Tensor:
     T = check_combine_args(cfg, y_perm, row_of_slot, topk_w)
     dev = y_perm.device
-    y = torch.empty((T, cfg.hidden_size), dtype=y_perm.dtype, device=dev)
+    y = torch.empty((T, cfg.hidden_size), dtype=out_dtype(cfg), device=dev)
     with torch.cuda.device(dev):
         _check(_lib.load().moe_combine(ctypes.byref(cfg), T, _p(y_perm), _p(row_of_slot), _p(topk_w), _p(y),
                                        _stream(dev)), "moe_combine")
@@ -290,7 +297,7 @@ def layer_forward(cfg: MoeConfig, x: torch.Tensor, w_router: torch.Tensor, b_rou
     T = check_layer_args(cfg, x, w_router, b_router, None if _weights_checked else weights, y, topk_ids, topk_w)
     dev = x.device
     if y is None:
-        y = torch.empty((T, cfg.hidden_size), dtype=x.dtype, device=dev)
+        y = torch.empty((T, cfg.hidden_size), dtype=out_dtype(cfg), device=dev)
     if ws is None:
         ws = torch.empty(max(workspace_size(cfg, T), 16), dtype=torch.uint8, device=dev)
     elif ws.device != dev:
@@ -340,9 +347,9 @@ def glm_expert_weights_from(d: Dict[str, torch.Tensor]) -> ExpertWeights:
     return ExpertWeights(d["w_gate"], d["w_up"], d["w_down"], None, None, None)
 
 
-def glm_config_from_spec(spec) -> MoeConfig:
+def glm_config_from_spec(spec, y_f32: bool = False) -> MoeConfig:
     """Config of a ``workloads.GlmLayerSpec`` (the SwiGLU limit and alpha are not used by the variant)."""
-    return make_config(spec.D, spec.F, spec.E, spec.k, dtype=spec.dtype)
+    return make_config(spec.D, spec.F, spec.E, spec.k, dtype=spec.dtype, y_f32=y_f32)
 
 
 def check_glm_args(cfg: MoeConfig, params: GlmParams, x, w_router, weights: Optional[ExpertWeights] = None,
@@ -371,7 +378,7 @@ def check_glm_args(cfg: MoeConfig, params: GlmParams, x, w_router, weights: Opti
         _want("w_up", weights.w_up, (E, F, D), dt, dev)
         _want("w_down", weights.w_down, (E, D, F), dt, dev)
     if y is not None:
-        _want("y", y, (T, D), dt, dev)
+        _want("y", y, (T, D), out_dtype(cfg), dev)
     if topk_ids is not None:
         _want("topk_ids", topk_ids, (T, k), torch.int32, dev)
     if topk_w is not None:
@@ -410,7 +417,7 @@ def glm_layer_forward(cfg: MoeConfig, params: GlmParams, x: torch.Tensor, w_rout
     T = check_glm_args(cfg, params, x, w_router, weights, y, topk_ids, topk_w)
     dev = x.device
     if y is None:
-        y = torch.empty((T, cfg.hidden_size), dtype=x.dtype, device=dev)
+        y = torch.empty((T, cfg.hidden_size), dtype=out_dtype(cfg), device=dev)
     if ws is None:
         ws = torch.empty(max(glm_workspace_size(cfg, params, T), 16), dtype=torch.uint8, device=dev)
     elif ws.device != dev:
@@ -469,7 +476,7 @@ class MoELayer:
         ``x`` holds at that time.  Removes host launch overhead (decode sizes).
         """
         if y is None:
-            y = torch.empty((x.shape[0], self.cfg.hidden_size), dtype=x.dtype, device=x.device)
+            y = torch.empty((x.shape[0], self.cfg.hidden_size), dtype=out_dtype(self.cfg), device=x.device)
         ws = self.workspace(x.shape[0])
         self(x, y=y, topk_ids=topk_ids, topk_w=topk_w)          # warm: per-device set-up outside capture
         torch.cuda.synchronize(x.device)
@@ -495,7 +502,7 @@ class MoELayer:
         dev = self.w_router.device
         T, D = xs_host[0].shape
         xd = [torch.empty((T, D), dtype=xs_host[0].dtype, device=dev) for _ in range(2)]
-        yd = [torch.empty((T, self.cfg.hidden_size), dtype=xs_host[0].dtype, device=dev) for _ in range(2)]
+        yd = [torch.empty((T, self.cfg.hidden_size), dtype=out_dtype(self.cfg), device=dev) for _ in range(2)]
         s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         cur = torch.cuda.current_stream(dev)
         for st in (s_in, s_run, s_out):

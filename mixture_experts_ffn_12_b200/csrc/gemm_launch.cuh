@@ -500,9 +500,10 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
     if ((e = make_tmap(&th, h, false, F, R, 0, kDecTok)) != cudaSuccess) return e;
     const int64_t units = (std::min<int64_t>(E, R) + R / kDecTok) * ((D + 127) / 128);
     if (slot_of_row != nullptr) {
-      // the split needs a 64-wide K block in each half: with F <= 64 the second half
-      // would be empty and add an accumulator that no MMA wrote
-      if (units <= L.num_sms && (F + 63) / 64 >= 2) {
+      // the split needs a K stage (kDecKBS 64-wide K blocks) in each half: with a single
+      // stage the second half would be empty and add an accumulator that no MMA wrote
+      constexpr int kStageK = 64 * kDecKBS;
+      if (units <= L.num_sms && (F + kStageK - 1) / kStageK >= 2) {
         // fewer units than SMs (T = 1: 4 experts x 23 feature blocks): split K in two,
         // each half adding its weighted partial into the zeroed fp32 rows
         const int64_t n = R * static_cast<int64_t>(D);

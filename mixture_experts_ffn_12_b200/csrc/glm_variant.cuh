@@ -100,17 +100,22 @@ __global__ void __launch_bounds__(256) glm_topk_kernel(const float* __restrict__
 }
 
 // The shared expert's one group: rows [0, T).
-__global__ void glm_shared_off_kernel(int32_t* __restrict__ off, int Tn) {
+__global__ void glm_shared_off_kernel(int32_t* __restrict__ off, int32_t* __restrict__ ident,
+                                      float* __restrict__ ones, int Tn) {
   pdl_enter();
-  if (threadIdx.x == 0) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
     off[0] = 0;
     off[1] = Tn;
   }
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < Tn; i += gridDim.x * blockDim.x) {
+    ident[i] = i;
+    ones[i] = 1.0f;
+  }
 }
 
-// y[t] = sum_j ys[t*k + j] (fp32, slot order) + y_shared[t] (dtype; may be null).
+// y[t] = sum_j ys[t*k + j] (fp32, slot order) + y_shared[t] (fp32; may be null), stored as T.
 template <typename T>
-__global__ void combine_slots_shared_kernel(const float* __restrict__ ys, const T* __restrict__ y_shared, int Tn,
+__global__ void combine_slots_shared_kernel(const float* __restrict__ ys, const float* __restrict__ y_shared, int Tn,
                                             int k, int D, T* __restrict__ y) {
   pdl_enter();
   const int nv = D / 8;
@@ -128,7 +133,7 @@ __global__ void combine_slots_shared_kernel(const float* __restrict__ ys, const 
     }
     if (y_shared != nullptr) {
       float v[8];
-      load8<T>(y_shared + static_cast<size_t>(t) * D + c, v);
+      load8<float>(y_shared + static_cast<size_t>(t) * D + c, v);
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] += v[q];
     }
@@ -168,20 +173,23 @@ cudaError_t glm_router(const Launch& L, bool bf16, int64_t T, int D, int E, int 
   return cudaGetLastError();
 }
 
-cudaError_t glm_shared_off(const Launch& L, int64_t T, int32_t* off) {
-  pdl_launch(glm_shared_off_kernel, dim3(1), dim3(32), 0, L.stream, off, static_cast<int>(T));
+// The shared expert as one group of T rows: offsets [0, T), and an identity slot map with
+// unit weights so that its down projection writes fp32 rows through the scatter epilogue.
+cudaError_t glm_shared_off(const Launch& L, int64_t T, int32_t* off, int32_t* ident, float* ones) {
+  const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((T + 255) / 256, int64_t(L.num_sms))));
+  pdl_launch(glm_shared_off_kernel, dim3(blocks), dim3(256), 0, L.stream, off, ident, ones, static_cast<int>(T));
   count_launch();
   return cudaGetLastError();
 }
 
-cudaError_t combine_slots_shared(const Launch& L, bool bf16, int64_t T, int D, int k, const void* ys,
+cudaError_t combine_slots_shared(const Launch& L, bool out_bf16, int64_t T, int D, int k, const void* ys,
                                  const void* y_shared, void* y) {
   if (T == 0) return cudaSuccess;
   const int64_t items = T * (D / 8);
   const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((items + 255) / 256, int64_t(L.num_sms) * 16)));
-  if (bf16)
+  if (out_bf16)
     pdl_launch(combine_slots_shared_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, L.stream,
-               static_cast<const float*>(ys), static_cast<const __nv_bfloat16*>(y_shared), static_cast<int>(T), k, D,
+               static_cast<const float*>(ys), static_cast<const float*>(y_shared), static_cast<int>(T), k, D,
                static_cast<__nv_bfloat16*>(y));
   else
     pdl_launch(combine_slots_shared_kernel<float>, dim3(blocks), dim3(256), 0, L.stream,
@@ -190,5 +198,4 @@ cudaError_t combine_slots_shared(const Launch& L, bool bf16, int64_t T, int D, i
   count_launch();
   return cudaGetLastError();
 }
-
 }  // namespace moe

@@ -55,11 +55,11 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
                         const int32_t* expert_off, const ExpertWeights& w, const int32_t* slot_of_row,
                         const float* topk_w, void* out);
 
-// y[t] = sum_j w[t,j] * y_perm[row_of_slot[t,j]]
-cudaError_t combine_gather(const Launch& L, bool bf16, int64_t T, int D, int k, const void* y_perm,
+// y[t] = sum_j w[t,j] * y_perm[row_of_slot[t,j]]   (y_perm in dtype; y in dtype, or fp32 if out_f32)
+cudaError_t combine_gather(const Launch& L, bool bf16, bool out_f32, int64_t T, int D, int k, const void* y_perm,
                            const int32_t* row_of_slot, const float* w, void* y);
-// y[t] = sum_j ys[t*k + j]   (ys fp32, y dtype)
-cudaError_t combine_slots(const Launch& L, bool bf16, int64_t T, int D, int k, const void* ys, void* y);
+// y[t] = sum_j ys[t*k + j]   (ys fp32; y bf16 if out_bf16, else fp32)
+cudaError_t combine_slots(const Launch& L, bool out_bf16, int64_t T, int D, int k, const void* ys, void* y);
 
 // The same two projections with MXFP4 expert weights, dequantised inside the GEMM mainloop.
 // The kernels read the E8M0 scales from a copy relaid as [E][ceil(K/64)][N][2]

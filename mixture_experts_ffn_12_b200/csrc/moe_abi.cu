@@ -50,9 +50,13 @@ moe_status_t check_cfg(const moe_config_t* c) {
   if (D % mult != 0 || F % mult != 0) return MOE_ERR_INVALID_ARG;
   if (!std::isfinite(c->swiglu_limit) || !(c->swiglu_limit > 0.0f) || !std::isfinite(c->swiglu_alpha))
     return MOE_ERR_INVALID_ARG;
+  if (c->y_f32 != 0 && c->y_f32 != 1) return MOE_ERR_INVALID_ARG;
   if (c->wfmt == MOE_W_MXFP4 && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
+
+// the layer output is bf16 only for a bf16 layer without y_f32
+bool out_bf16(const moe_config_t* c) { return c->dtype == MOE_BF16 && c->y_f32 == 0; }
 
 bool check_T(int64_t T, int k) { return T >= 0 && T * k < (int64_t(1) << 31); }
 
@@ -193,19 +197,57 @@ moe_status_t run_experts(const moe_config_t* c, const Launch& L, int64_t T, cons
 constexpr size_t kNoAllocWords = 65536;
 static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocWords];
 
-// Host code cannot use g_permute_scratch's name as a device address, so the
-// address is looked up once per device (with that device current) and cached.
-int32_t* permute_scratch_address(int dev) {
-  static std::mutex mu;
-  static int32_t* addr[64] = {};
-  if (dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> g(mu);
-  if (addr[dev] == nullptr) {
+// Host code cannot use g_permute_scratch's name as a device address: the address
+// is looked up with cudaGetSymbolAddress in the current CUDA context.  It belongs
+// to that context, so lookups are cached per context, keyed by the context's unique
+// id (cuCtxGetId, never reused within a process): a context the caller made current
+// itself, or the new primary context after a cudaDeviceReset, gets its own lookup.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<int32_t*>(p);
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+int32_t* permute_scratch_address() {
+  struct Entry {
+    unsigned long long ctx_id;
+    int32_t* addr;
+  };
+  constexpr int kSlots = 64;
+  static Entry cache[kSlots] = {};
+  static int next = 0;
+  static std::mutex mu;
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);   // false before the runtime made a context current
+  std::lock_guard<std::mutex> g(mu);
+  if (have_id)
+    for (const Entry& e : cache)
+      if (e.addr != nullptr && e.ctx_id == id) return e.addr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) return nullptr;
+  if (have_id || current_context_id(&id)) {
+    cache[next] = Entry{id, static_cast<int32_t*>(p)};
+    next = (next + 1) % kSlots;
   }
-  return addr[dev];
+  return static_cast<int32_t*>(p);
 }
 
 // ---------------------------------------------------------------------------
@@ -222,7 +264,7 @@ moe_status_t check_glm(const moe_config_t* c, const moe_glm_params_t* p) {
 }
 
 struct GlmLayout {
-  size_t ids, w, off, ros, sor, pscr, xperm, ys, h, rpart, zb, soff, hs, ysh, total;
+  size_t ids, w, off, ros, sor, pscr, xperm, ys, h, rpart, zb, soff, sid, sone, hs, ysh, total;
 };
 
 GlmLayout glm_layout(const moe_config_t* c, const moe_glm_params_t* p, int64_t T) {
@@ -253,8 +295,10 @@ GlmLayout glm_layout(const moe_config_t* c, const moe_glm_params_t* p, int64_t T
   L.zb = take(zb * es);
   if (Fs > 0) {
     L.soff = take(2 * 4);
+    L.sid = take(size_t(T) * 4);
+    L.sone = take(size_t(T) * 4);
     L.hs = take(size_t(T) * Fs * es);
-    L.ysh = take(size_t(T) * D * es);
+    L.ysh = take(size_t(T) * D * 4);
   }
   L.total = o;
   return L;
@@ -344,9 +388,7 @@ moe_status_t moe_permute_noalloc(const moe_config_t* cfg, int64_t T, const int32
     if (x != nullptr && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
     if (moe::permute_scratch_words(T, cfg->num_local_experts) > kNoAllocWords) return MOE_ERR_UNSUPPORTED;
   }
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  int32_t* scratch = permute_scratch_address(dev);
+  int32_t* scratch = permute_scratch_address();
   if (scratch == nullptr) return MOE_ERR_CUDA;
   Launch L;
   if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
@@ -380,8 +422,8 @@ moe_status_t moe_combine(const moe_config_t* cfg, int64_t T, const void* y_perm,
   if (!ptr_ok(y_perm) || !ptr_ok(row_of_slot) || !ptr_ok(topk_w) || !ptr_ok(y)) return MOE_ERR_INVALID_ARG;
   Launch L;
   if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
-  return cuda_status(moe::combine_gather(L, cfg->dtype == MOE_BF16, T, cfg->hidden_size, cfg->num_experts_per_tok,
-                                         y_perm, row_of_slot, topk_w, y));
+  return cuda_status(moe::combine_gather(L, cfg->dtype == MOE_BF16, cfg->y_f32 != 0, T, cfg->hidden_size,
+                                         cfg->num_experts_per_tok, y_perm, row_of_slot, topk_w, y));
 }
 
 moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x, const void* w_router,
@@ -425,7 +467,7 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x
   s = run_experts(cfg, L, T, xperm, eoff, weights, h, ys, sor, w, ffn);
   if (s != MOE_OK) return s;
   stage_mark(ST_COMBINE, true, L.stream);
-  s = cuda_status(moe::combine_slots(L, bf16, T, D, k, ys, y));
+  s = cuda_status(moe::combine_slots(L, out_bf16(cfg), T, D, k, ys, y));
   stage_mark(ST_COMBINE, false, L.stream);
   return s;
 }
@@ -556,13 +598,15 @@ moe_status_t moe_glm_layer_forward(const moe_config_t* cfg, const moe_glm_params
     sw.b_gate = zb;
     sw.b_up = zb;
     sw.b_down = zb;
-    if (moe::glm_shared_off(L, T, soff) != cudaSuccess) return MOE_ERR_CUDA;
+    int32_t* sid = reinterpret_cast<int32_t*>(base + LY.sid);
+    float* sone = reinterpret_cast<float*>(base + LY.sone);
+    if (moe::glm_shared_off(L, T, soff, sid, sone) != cudaSuccess) return MOE_ERR_CUDA;
     if (moe::expert_gateup(L, bf16, T, D, Fs, 1, x, soff, sw, kInf, 1.0f, hs, -kInf) != cudaSuccess)
       return MOE_ERR_CUDA;
-    if (moe::expert_down(L, bf16, T, D, Fs, 1, hs, soff, sw, nullptr, nullptr, ysh) != cudaSuccess)
-      return MOE_ERR_CUDA;
+    // fp32 rows (identity slots, unit weights): the shared output is rounded once, with the sum
+    if (moe::expert_down(L, bf16, T, D, Fs, 1, hs, soff, sw, sid, sone, ysh) != cudaSuccess) return MOE_ERR_CUDA;
   }
-  return cuda_status(moe::combine_slots_shared(L, bf16, T, D, k, ys, ysh, y));
+  return cuda_status(moe::combine_slots_shared(L, out_bf16(cfg), T, D, k, ys, ysh, y));
 }
 
 }  // extern "C"

@@ -600,9 +600,9 @@ cudaError_t permute(const Launch& L, bool bf16, int64_t T, int D, int E, int k, 
 // ---------------------------------------------------------------------------
 // combine
 // ---------------------------------------------------------------------------
-template <typename T>
+template <typename T, typename TO>
 __global__ void combine_gather_kernel(const T* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
-                                      const float* __restrict__ w, int Tn, int k, int D, T* __restrict__ y) {
+                                      const float* __restrict__ w, int Tn, int k, int D, TO* __restrict__ y) {
   pdl_enter();
   const int nv = D / 8;
   const int64_t total = static_cast<int64_t>(Tn) * nv;
@@ -624,7 +624,7 @@ __global__ void combine_gather_kernel(const T* __restrict__ y_perm, const int32_
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] = fmaf(wt, v[q], acc[q]);
     }
-    store8<T>(y + static_cast<size_t>(t) * D + c, acc);
+    store8<TO>(y + static_cast<size_t>(t) * D + c, acc);
   }
 }
 
@@ -653,30 +653,34 @@ static int elementwise_blocks(const Launch& L, int64_t items) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(L.num_sms) * 16)));
 }
 
-cudaError_t combine_gather(const Launch& L, bool bf16, int64_t T, int D, int k, const void* y_perm,
+cudaError_t combine_gather(const Launch& L, bool bf16, bool out_f32, int64_t T, int D, int k, const void* y_perm,
                            const int32_t* row_of_slot, const float* w, void* y) {
   if (T == 0) return cudaSuccess;
   const int blocks = elementwise_blocks(L, T * (D / 8));
-  if (bf16)
-    pdl_launch(combine_gather_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, L.stream, 
-        static_cast<const __nv_bfloat16*>(y_perm), row_of_slot, w, static_cast<int>(T), k, D,
-        static_cast<__nv_bfloat16*>(y));
+  const int Ti = static_cast<int>(T);
+  if (bf16 && !out_f32)
+    pdl_launch(combine_gather_kernel<__nv_bfloat16, __nv_bfloat16>, dim3(blocks), dim3(256), 0, L.stream,
+               static_cast<const __nv_bfloat16*>(y_perm), row_of_slot, w, Ti, k, D, static_cast<__nv_bfloat16*>(y));
+  else if (bf16)
+    pdl_launch(combine_gather_kernel<__nv_bfloat16, float>, dim3(blocks), dim3(256), 0, L.stream,
+               static_cast<const __nv_bfloat16*>(y_perm), row_of_slot, w, Ti, k, D, static_cast<float*>(y));
   else
-    pdl_launch(combine_gather_kernel<float>, dim3(blocks), dim3(256), 0, L.stream, static_cast<const float*>(y_perm), row_of_slot, w,
-                                                              static_cast<int>(T), k, D, static_cast<float*>(y));
+    pdl_launch(combine_gather_kernel<float, float>, dim3(blocks), dim3(256), 0, L.stream,
+               static_cast<const float*>(y_perm), row_of_slot, w, Ti, k, D, static_cast<float*>(y));
   count_launch();
   return cudaGetLastError();
 }
 
-cudaError_t combine_slots(const Launch& L, bool bf16, int64_t T, int D, int k, const void* ys, void* y) {
+// y in bf16 (out_bf16) or fp32; the fp32 sums are the same either way
+cudaError_t combine_slots(const Launch& L, bool out_bf16, int64_t T, int D, int k, const void* ys, void* y) {
   if (T == 0) return cudaSuccess;
   const int blocks = elementwise_blocks(L, T * (D / 8));
-  if (bf16)
-    pdl_launch(combine_slots_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, L.stream, 
-        static_cast<const float*>(ys), static_cast<int>(T), k, D, static_cast<__nv_bfloat16*>(y));
+  if (out_bf16)
+    pdl_launch(combine_slots_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, L.stream,
+               static_cast<const float*>(ys), static_cast<int>(T), k, D, static_cast<__nv_bfloat16*>(y));
   else
-    pdl_launch(combine_slots_kernel<float>, dim3(blocks), dim3(256), 0, L.stream, static_cast<const float*>(ys), static_cast<int>(T),
-                                                             k, D, static_cast<float*>(y));
+    pdl_launch(combine_slots_kernel<float>, dim3(blocks), dim3(256), 0, L.stream, static_cast<const float*>(ys),
+               static_cast<int>(T), k, D, static_cast<float*>(y));
   count_launch();
   return cudaGetLastError();
 }

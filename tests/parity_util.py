@@ -42,23 +42,42 @@ def layer_for(spec: W.LayerSpec, seed: int = 0, experts: bool = True):
     return layer
 
 
-def check_output(got: np.ndarray, ref: np.ndarray, tol: float, bf16_out: bool) -> float:
-    """Layer output check: |got - ref| <= tol * RMS(ref) + (output rounding) per element.
+def check_output(got: np.ndarray, ref: np.ndarray, tol: float) -> float:
+    """Layer output check, the acceptance bound as written: max |got - ref| <= tol * RMS(ref).
 
-    The output is stored in the activation dtype.  Rounding the exact fp64
-    result to bf16 moves an element by up to half an ulp, <= 2^-8 |ref|, which
-    on large-magnitude elements is already close to 2e-2 of the RMS (for the
-    GPT-OSS-120B-shaped layer: 1.75e-2 on the sampled tokens, 2^-8 x max|y|/RMS
-    = 2.3e-2 in the worst case), so that rounding is allowed on top of the bound.
-    Returns the raw max |got - ref| / RMS(ref) for the record.
+    ``got`` is the fp32 layer output (the layer's y_f32 option): for a bf16 layer,
+    rounding even the exact fp64 result to bf16 moves the largest elements by up
+    to 2^-8 |y|, which reaches 2e-2 of the RMS on the GPT-OSS-120B-shaped layer
+    (max |y| / RMS = 6.7) -- no bf16-stored output can meet the bound there, so
+    the bound is asserted on the fp32 output and the bf16 output is checked to be
+    exactly its rounding (``check_rounding``).  Returns the max error / RMS.
     """
     rms = float(np.sqrt(np.mean(np.square(ref))))
-    allow = (2.0 ** -8 if bf16_out else 2.0 ** -23) * np.abs(ref)
-    excess = np.abs(got - ref) - (tol * rms + allow)
     raw = float(np.max(np.abs(got - ref))) / max(rms, 1e-30)
-    assert np.all(excess <= 0), f"max excess {excess.max():.3e}; raw max err / RMS = {raw:.3e}"
-    print(f"max err / RMS = {raw:.3e}")
+    print(f"max err / RMS = {raw:.3e} (bound {tol:g})")
+    assert raw <= tol, f"max |y - y_ref| / RMS = {raw:.4e} > {tol:g}"
     return raw
+
+
+def check_rounding(y_out, y32, ref: np.ndarray = None) -> None:
+    """The layer output in its dtype is the round-to-nearest-even of the fp32 output, bit for bit.
+
+    y_out, y32: torch tensors of the same layer call made with and without y_f32.
+    For the record, prints the max error / RMS of the bf16 output and of the exact
+    result rounded to bf16 (both include the same storage rounding).
+    """
+    import torch
+    if y_out.dtype == torch.float32:
+        assert torch.equal(y_out, y32)
+        return
+    want = W.f32_to_bf16_bits(y32.cpu().numpy())
+    got = y_out.cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want), "bf16 output is not the rounding of the fp32 output"
+    if ref is not None:
+        rms = float(np.sqrt(np.mean(np.square(ref))))
+        exact_rounded = W.bf16_bits_to_f32(W.f32_to_bf16_bits(ref.astype(np.float32))).astype(np.float64)
+        print(f"bf16 output: max err / RMS = {np.max(np.abs(f64(y_out) - ref)) / rms:.3e}; "
+              f"exact result rounded to bf16: {np.max(np.abs(exact_rounded - ref)) / rms:.3e}")
 
 
 def rel_rms(got: np.ndarray, ref: np.ndarray) -> float:

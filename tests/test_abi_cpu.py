@@ -32,7 +32,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_struct_layout_matches_header():
-    assert ctypes.sizeof(_lib.MoeConfig) == 32
+    assert ctypes.sizeof(_lib.MoeConfig) == 36
+    assert _lib.MoeConfig.y_f32.offset == 32
     assert ctypes.sizeof(_lib.MoeExpertWeights) == 9 * ctypes.sizeof(ctypes.c_void_p)
     # int32, float, four pointers, int32 (+ tail padding to pointer alignment)
     assert ctypes.sizeof(_lib.MoeGlmParams) == 48
@@ -48,7 +49,7 @@ def cfg(**kw):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2 == _lib.ABI_VERSION
     for code in range(7):
         assert lib.moe_status_string(code).startswith(b"MOE_")
     assert b"unknown" in lib.moe_status_string(99)
@@ -72,6 +73,10 @@ def test_version_and_status_strings(lib):
     (dict(swiglu_limit=float("nan")), _lib.MOE_ERR_INVALID_ARG),
     (dict(dtype=7), _lib.MOE_ERR_INVALID_ARG),
     (dict(wfmt=3), _lib.MOE_ERR_INVALID_ARG),
+    (dict(y_f32=1), _lib.MOE_OK),
+    (dict(y_f32=1, dtype=_lib.MOE_F32), _lib.MOE_OK),
+    (dict(y_f32=2), _lib.MOE_ERR_INVALID_ARG),
+    (dict(y_f32=-1), _lib.MOE_ERR_INVALID_ARG),
 ])
 def test_config_check(lib, kw, want):
     assert lib.moe_config_check(ctypes.byref(cfg(**kw))) == want
@@ -153,9 +158,11 @@ def test_glm_workspace_sizes(lib):
     assert base < R * D * 4 + R * F * 2 + 4 * R * 4 + E * F * 2 + 64 * 1024 * 1024
     p = ctypes.c_void_p(0x10000).value
     shared = glm_params(ws_gate=p, ws_up=p, ws_down=p, shared_intermediate_size=1408)
-    # a shared expert adds its offsets, [T, Fs] and [T, D] in bf16
+    # a shared expert adds its offsets, identity slots and unit weights [T], [T, Fs] in bf16
+    # and its fp32 output rows [T, D]
     extra = lib.moe_glm_workspace_size(ctypes.byref(c), ctypes.byref(shared), T) - base
-    assert T * 1408 * 2 + T * D * 2 <= extra <= T * 1408 * 2 + T * D * 2 + 4 * 256
+    want = T * 4 * 2 + T * 1408 * 2 + T * D * 4
+    assert want <= extra <= want + 6 * 256
     assert lib.moe_glm_workspace_size(ctypes.byref(c), None, T) == _lib.SIZE_INVALID
     assert lib.moe_glm_workspace_size(ctypes.byref(c), ctypes.byref(glm_params(shared_intermediate_size=24)), T) \
         == _lib.SIZE_INVALID

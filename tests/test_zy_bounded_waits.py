@@ -11,7 +11,7 @@ import pytest
 
 import workloads as W
 from oracle import moe_oracle as O
-from parity_util import check_ids, check_output, f64, layer_for, tol_for
+from parity_util import check_ids, check_output, check_rounding, f64, layer_for, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -39,11 +39,15 @@ def test_timeout_is_reported_and_context_survives():
         api.set_wait_limit_ns(0)
         api.set_expert_gemm_variant(0)
     assert status == _lib.MOE_ERR_TIMEOUT
-    # the context is intact: a normal call is right
+    # the context is intact: a normal call is right (fp32 output within the bound, and the
+    # bf16 output of a second call its rounding)
     ids = torch.empty((spec.T, spec.k), dtype=torch.int32, device="cuda")
-    y = api.layer_forward(cfg, d["x"], d["w_router"], d["b_router"], ew, topk_ids=ids)
+    y32 = api.layer_forward(api.config_from_spec(spec, y_f32=True), d["x"], d["w_router"], d["b_router"], ew,
+                            topk_ids=ids)
+    y = api.layer_forward(cfg, d["x"], d["w_router"], d["b_router"], ew)
     torch.cuda.synchronize()
     assert api.last_device_error() == _lib.MOE_OK
     ref = O.layer_tokens(layer, np.arange(spec.T), spec.k, spec.limit, spec.alpha)
     check_ids(ids.cpu().numpy(), ref["ids"], ref["logits"])
-    check_output(f64(y), ref["y"], tol_for(spec), True)
+    check_output(f64(y32), ref["y"], tol_for(spec))
+    check_rounding(y, y32, ref["y"])

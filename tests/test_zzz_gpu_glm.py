@@ -3,15 +3,16 @@
 Source of the variant: "Ollama glm4_moe_lite.go" (MoEGate.Forward, SwitchMLP.Forward,
 SharedExperts.Forward, MoE.Forward).  Bit-exact: the chosen expert sets (and their
 order where the corrected scores are separated).  Routing weights within 2e-5 (they
-include routed_scaling_factor).  Layer output within 2e-2 of the output's RMS plus
-its own storage rounding, the bound of the GPT-OSS layer.
+include routed_scaling_factor).  Each layer call runs with the output in the layer
+dtype and in fp32 (y_f32): the fp32 output within 2e-2 of the output's RMS, the
+bound of the GPT-OSS layer as written, and the dtype output exactly its rounding.
 """
 import numpy as np
 import pytest
 
 import workloads as W
 from oracle import glm_moe as G
-from parity_util import TOL_W, TOL_Y, check_ids, check_output, f64
+from parity_util import TOL_W, TOL_Y, check_ids, check_output, check_rounding, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -48,16 +49,27 @@ def _layer(spec):
 
 
 def _run(api, spec, layer):
+    """The layer with y in its dtype and with y in fp32: (y, y32, ids, w)."""
     d = api.upload_layer(layer)
-    cfg = api.glm_config_from_spec(spec)
     params = api.glm_params_from(spec, d)
-    ids = torch.empty((spec.T, spec.k), dtype=torch.int32, device="cuda")
-    w = torch.empty((spec.T, spec.k), dtype=torch.float32, device="cuda")
-    y = api.glm_layer_forward(cfg, params, d["x"], d["w_router"], api.glm_expert_weights_from(d),
-                              topk_ids=ids, topk_w=w)
-    torch.cuda.synchronize()
-    assert api.last_device_error() == 0
-    return y, ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+    out = []
+    for y_f32 in (False, True):
+        cfg = api.glm_config_from_spec(spec, y_f32=y_f32)
+        ids = torch.empty((spec.T, spec.k), dtype=torch.int32, device="cuda")
+        w = torch.empty((spec.T, spec.k), dtype=torch.float32, device="cuda")
+        y = api.glm_layer_forward(cfg, params, d["x"], d["w_router"], api.glm_expert_weights_from(d),
+                                  topk_ids=ids, topk_w=w)
+        torch.cuda.synchronize()
+        assert api.last_device_error() == 0
+        out.append((y, ids, w))
+    (y, ids, w), (y32, ids32, w32) = out
+    assert torch.equal(ids, ids32) and torch.equal(w, w32)
+    return y, y32, ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+
+
+def _check_layer(y, y32, ref_y, tol):
+    check_output(f64(y32), ref_y, tol)
+    check_rounding(y, y32, ref_y)
 
 
 def _check_weights(gid, gw, rid, rw):
@@ -69,11 +81,11 @@ def _check_weights(gid, gw, rid, rw):
 @pytest.mark.parametrize("spec", SPECS, ids=lambda s: s.name)
 def test_glm_layer_forward(api, spec):
     layer = _layer(spec)
-    y, gid, gw = _run(api, spec, layer)
+    y, y32, gid, gw = _run(api, spec, layer)
     ref = G.layer_forward(layer, spec.k, spec.norm_topk_prob, spec.routed_scaling_factor)
     check_ids(gid, ref["ids"], ref["chosen_by"])
     _check_weights(gid, gw, ref["ids"], ref["w"])
-    check_output(f64(y), ref["y"], TOL_Y[spec.dtype], spec.dtype == "bf16")
+    _check_layer(y, y32, ref["y"], TOL_Y[spec.dtype])
 
 
 @pytest.mark.parametrize("spec", [GLM_TC_ROUTER, GLM_F32, GLM_K1, GLM_MANY], ids=lambda s: s.name)
@@ -100,12 +112,12 @@ def test_glm_each_gemm_variant(api, variant):
     layer = _layer(spec)
     api.set_expert_gemm_variant(variant)
     try:
-        y, gid, _ = _run(api, spec, layer)
+        y, y32, gid, _ = _run(api, spec, layer)
     finally:
         api.set_expert_gemm_variant(0)
     ref = G.layer_forward(layer, spec.k, spec.norm_topk_prob, spec.routed_scaling_factor)
     check_ids(gid, ref["ids"], ref["chosen_by"])
-    check_output(f64(y), ref["y"], TOL_Y["bf16"], True)
+    _check_layer(y, y32, ref["y"], TOL_Y["bf16"])
 
 
 def test_glm_zero_tokens(api):

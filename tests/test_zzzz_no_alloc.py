@@ -59,6 +59,37 @@ def test_noalloc_permute_matches_workspace_version():
     assert int(first[0][-1]) == 9000 * 4 and int(second[0][-1]) == 300 * 4
 
 
+def test_noalloc_permute_takes_no_device_memory():
+    """A call (after the first one on this device) leaves the device's free memory unchanged."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from mixture_experts_ffn_12_b200 import _lib, build
+    build.build()
+    lib = _lib.load()
+    T, E, k, D = 4096, 32, 4, 64
+    rng = np.random.default_rng(3)
+    ids = torch.from_numpy(np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)).cuda()
+    x = torch.zeros((T, D), dtype=torch.bfloat16, device="cuda")
+    outs = (torch.empty(E + 1, dtype=torch.int32, device="cuda"), torch.empty(T * k, dtype=torch.int32, device="cuda"),
+            torch.empty(T * k, dtype=torch.int32, device="cuda"),
+            torch.empty((T * k, D), dtype=torch.bfloat16, device="cuda"))
+    cfg = _lib.MoeConfig(D, 64, E, k, 7.0, 1.702, _lib.MOE_BF16, _lib.MOE_W_DENSE)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+
+    def call():
+        assert lib.moe_permute_noalloc(ctypes.byref(cfg), T, p(ids), p(x), *(p(o) for o in outs), stream) == \
+            _lib.MOE_OK
+        torch.cuda.synchronize()
+
+    call()                                   # the first call in this context looks up the array
+    free_before, _ = torch.cuda.mem_get_info()
+    call()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert lib.moe_last_device_error() == _lib.MOE_OK
+    assert free_after == free_before
+
+
 def test_noalloc_permute_rejects_sizes_beyond_its_array():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
