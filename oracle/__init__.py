@@ -14,10 +14,12 @@ Two levels:
 
 ``glm_moe`` is the O1 oracle of the layer's GLM4-MoE-Lite variant (sigmoid
 router with a selection-only correction bias, SiLU experts, a shared expert);
-``brute`` holds its scalar-loop counterpart.
+``mx_act`` the O1 oracle of the MXFP4 layer with its activations in MXFP8 (the
+block-scaled numerics variant); ``brute`` holds the scalar-loop counterparts of
+both.
 
-Every function is pinned by ``tests/test_oracle_pins.py`` (brute force, closed
+Every function is pinned by ``tests/test_oracle_pins*.py`` (brute force, closed
 forms, invariants, hand-worked values in ``tests/golden/``).  No function here
 is "parity unpinned".
 """
-from . import moe_oracle, brute, glm_moe  # noqa: F401
+from . import moe_oracle, brute, glm_moe, mx_act  # noqa: F401

@@ -246,3 +246,71 @@ def glm_layer_token(layer, t: int, k: int, norm_topk_prob: bool, routed_scaling_
         for d in range(D):
             y[d] += o[d]
     return dict(logits=lg, ids=ids, w=w, y=y)
+
+
+# --------------------------------------------------------------------------- #
+# MXFP8 activations (the block-scaled numerics variant, pins ``mx_act``)
+# --------------------------------------------------------------------------- #
+def e4m3_table() -> List[Tuple[int, float]]:
+    """(code, value) of every finite E4M3 code, built bit field by bit field."""
+    out = []
+    for code in range(256):
+        s = -1.0 if code & 0x80 else 1.0
+        e = (code >> 3) & 0xF
+        m = code & 0x7
+        if e == 0xF and m == 0x7:
+            continue                                   # NaN
+        if e == 0:
+            val = s * m * 2.0 ** -9
+        else:
+            val = s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+        out.append((code, val))
+    return out
+
+
+def e4m3_nearest(v: float) -> float:
+    """The finite E4M3 value nearest to v (ties: the code with an even mantissa), by search."""
+    best, best_code = None, None
+    for code, val in e4m3_table():
+        if best is None or abs(val - v) < abs(best - v) or (
+                abs(val - v) == abs(best - v) and (code & 1) == 0 and (best_code & 1) == 1):
+            best, best_code = val, code
+    return best + 0.0   # -0.0 -> 0.0
+
+
+def mx8_exponent(amax: float) -> int:
+    """Smallest X in [-127, 127] with amax <= 448 * 2^X (searching upwards)."""
+    for X in range(-127, 128):
+        if amax <= 448.0 * 2.0 ** X:
+            return X
+    return 127
+
+
+def mx8_row(v: Sequence[float]) -> List[float]:
+    """One row quantized to MXFP8 and dequantized, 32-element blocks."""
+    out = []
+    for b in range(0, len(v), 32):
+        blk = list(v[b:b + 32])
+        X = mx8_exponent(max(abs(t) for t in blk))
+        out.extend(e4m3_nearest(t / 2.0 ** X) * 2.0 ** X for t in blk)
+    return out
+
+
+def layer_token_mx8(layer, t: int, k: int, limit: float, alpha: float = 1.702) -> Dict[str, list]:
+    """One token through the layer with MXFP8 activations in both expert projections."""
+    logits = router_logits(layer, t)
+    ids, w = topk_bruteforce(logits, k)
+    x = mx8_row([value(v) for v in layer["x"][t]])
+    D = len(layer["b_down"][0])
+    y = [0.0] * D
+    for e, wt in zip(ids, w):
+        F = len(layer["b_gate"][e])
+        h = []
+        for f in range(F):
+            g = dot(x, weight_row(layer, "gate", e, f)) + value(layer["b_gate"][e][f])
+            u = dot(x, weight_row(layer, "up", e, f)) + value(layer["b_up"][e][f])
+            h.append(swiglu(g, u, limit, alpha))
+        hq = mx8_row(h)
+        for d in range(D):
+            y[d] += wt * (dot(hq, weight_row(layer, "down", e, d)) + value(layer["b_down"][e][d]))
+    return {"ids": ids, "w": w, "y": y}
