@@ -52,6 +52,8 @@ def parse_args():
     p.add_argument("--no-mxfp4", action="store_true", help="skip the MXFP4-weight layer")
     p.add_argument("--no-skewed", action="store_true", help="skip the GPT-OSS-120B-shaped skewed layer")
     p.add_argument("--no-glm", action="store_true", help="skip the GLM4-MoE-Lite variant layer")
+    p.add_argument("--h-split", action="store_true",
+                   help="keep the SwiGLU output as two bf16 halves between the expert GEMMs (h_split)")
     return p.parse_args()
 
 
@@ -65,8 +67,8 @@ def measured_peaks():
     return dict(bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, hbm_gbs=6650.0, source="fallback")
 
 
-def config_of(spec, n_gpus):
-    return {"workload": spec.name, "T_per_gpu": spec.T, "hidden_size": spec.D, "intermediate_size": spec.F,
+def config_of(spec, n_gpus, h_split=False):
+    return {"workload": spec.name, "h_split": h_split, "T_per_gpu": spec.T, "hidden_size": spec.D, "intermediate_size": spec.F,
             "num_local_experts": spec.E, "num_experts_per_tok": spec.k, "swiglu_limit": spec.limit,
             "expert_weights": spec.wfmt, "global_tokens": spec.T * n_gpus,
             "parallelism": f"dp{n_gpus} (independent replicas)",
@@ -226,7 +228,7 @@ def run_ours(args, rank, world, local_rank):
     if rank > 0:   # each replica routes its own tokens
         layer["x"] = W.make_layer(spec, seed=rank, with_experts=False)["x"]
     d = api.upload_layer(layer, dev)
-    cfg = api.config_from_spec(spec)
+    cfg = api.config_from_spec(spec, h_split=args.h_split)
     moe = api.MoELayer(cfg, d["w_router"], d["b_router"], api.expert_weights_from(d))
     x, T = d["x"], spec.T
     y = torch.empty_like(x)
@@ -306,6 +308,14 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1))
 
+    # the same layer with h kept as two bf16 halves between the expert GEMMs (the precise form)
+    hsplit = None
+    if not args.h_split and spec.dtype == "bf16" and spec.wfmt == "dense":
+        moe2 = api.MoELayer(api.config_from_spec(spec, h_split=True), d["w_router"], d["b_router"], moe.experts)
+        for _ in range(3):
+            moe2(x, y=y)
+        hsplit = {"ms_per_step": timed_steps(lambda: moe2(x, y=y), stream, max(10, K // 2))}
+        del moe2
     decode = decode_sweep(api, moe, spec, layer, dev, stream, max(20, K // 4)) if not args.no_decode else None
     mx = sk = glm = None
     extra = world == 1 and spec.name == W.GPTOSS20B_PREFILL.name
@@ -336,7 +346,7 @@ def run_ours(args, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if spec.dtype == "bf16" else "f32",
             "data": "synthetic (seeded random-init weights and activations of the GPT-OSS-20B MoE layer shape)",
-            "config": config_of(spec, world),
+            "config": config_of(spec, world, args.h_split),
             "tflops": flops / (ms_step / 1e3) / 1e12,
             "roofline": {"bound": "tensor", "kernel": "gateup_swiglu_gemm", "achieved": achieved,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
@@ -352,6 +362,8 @@ def run_ours(args, rank, world, local_rank):
             "gpu_launches": int(launches),
             "clocks": sampler.summary(),
         }
+        if hsplit is not None:
+            line["h_split"] = hsplit
         if decode is not None:
             line["decode"] = decode
         if mx is not None:
@@ -496,6 +508,12 @@ def skewed_sweep(api, dev, stream, steps):
     touched = int((cnt > 0).sum())
     ms = timed_steps(lambda: moe(x, y=y), stream, steps)
     stage = stage_times(lambda: moe(x, y=y), stream, min(steps, 10))
+    # the same layer with h kept as two bf16 halves (the down projection does twice the MMA work)
+    moe2 = api.MoELayer(api.config_from_spec(spec, h_split=True), d["w_router"], d["b_router"], moe.experts)
+    for _ in range(2):
+        moe2(x, y=y)
+    ms_split = timed_steps(lambda: moe2(x, y=y), stream, steps)
+    del moe2
     if api.last_device_error() != 0:
         raise RuntimeError("device error word set during the skewed-layer steps")
     flops = spec.expert_flops() + spec.router_flops()
@@ -505,7 +523,7 @@ def skewed_sweep(api, dev, stream, steps):
            "tflops": flops / (ms * 1e-3) / 1e12, "experts_touched": touched,
            "max_expert_rows": int(cnt.max()), "touched_weight_bytes": nbytes,
            "roofline_us": 1e3 * roof_ms, "frac": roof_ms / ms,
-           "stage_us": {k: 1e3 * v for k, v in stage.items()},
+           "stage_us": {k: 1e3 * v for k, v in stage.items()}, "us_per_step_h_split": 1e3 * ms_split,
            "weights": "expert weights drawn on the device (same law as the recipe); x and router from the recipe"}
     del moe, d
     torch.cuda.empty_cache()

@@ -98,6 +98,13 @@ typedef struct {
                                   layer the dtype output is exactly the round-to-nearest-even
                                   of this fp32 output).  Applies to moe_layer_forward,
                                   moe_combine and moe_glm_layer_forward. */
+  int32_t h_split;             /* 0: the SwiGLU output h is kept in dtype between the two expert
+                                  GEMMs.  1 (bf16 layers with dense weights): h is kept as two
+                                  bf16 halves, hi = bf16(h) and lo = bf16(h - hi), and the down
+                                  projection sums over both against the same weights (twice its
+                                  tensor-core work), so h carries about 16 significant bits
+                                  instead of 8.  No effect on fp32 layers; MOE_ERR_UNSUPPORTED
+                                  with MXFP4 weights or with expert-GEMM variant 4. */
 } moe_config_t;
 
 /* Expert parameters (device pointers).  Dense: w_* in dtype, s_* NULL.
@@ -136,7 +143,7 @@ MOE_API size_t moe_expert_ffn_workspace_size(const moe_config_t* cfg, int64_t T)
 
 /* Bytes of workspace moe_layer_forward needs for T tokens: routing ids and
  * weights, dispatch maps, permuted activations x_perm [T*k, D], the SwiGLU
- * output h [T*k, F], the weighted expert outputs [T*k, D] in fp32 (sharing
+ * output h [T*k, F] ([T*k, 2, F] with h_split), the weighted expert outputs [T*k, D] in fp32 (sharing
  * x_perm's space), plus what the sub-steps need.  (size_t)-1 if cfg is invalid. */
 MOE_API size_t moe_workspace_size(const moe_config_t* cfg, int64_t T);
 
@@ -191,7 +198,9 @@ MOE_API moe_status_t moe_permute_noalloc(const moe_config_t* cfg, int64_t T, con
 
 /* Per-expert FFN over the permuted rows (R = T*k):
  *   x_perm [R, D], expert_off [E+1] (as produced by moe_permute; read on the device)
- *   -> h [R, F]: clipped SwiGLU of the gate/up projections (+ biases),
+ *   -> h [R, F]: clipped SwiGLU of the gate/up projections (+ biases); with
+ *      cfg->h_split, h is [R, 2, F]: row r holds bf16(h[r]) then the bf16 rounding
+ *      of h[r] - bf16(h[r]),
  *      y_perm [R, D]: h Wd[e]^T + bd[e] for the expert e that owns each row.
  * Computed on the tcgen05 tensor cores with fp32 accumulation from bf16
  * operands (MXFP4 weights are decoded to bf16 in shared memory inside the GEMM

@@ -35,6 +35,7 @@ class MoeConfig(ctypes.Structure):
         ("dtype", ctypes.c_int32),
         ("wfmt", ctypes.c_int32),
         ("y_f32", ctypes.c_int32),
+        ("h_split", ctypes.c_int32),
     ]
 
 

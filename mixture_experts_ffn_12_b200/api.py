@@ -35,16 +35,18 @@ _DT = {"bf16": (_lib.MOE_BF16, torch.bfloat16), "f32": (_lib.MOE_F32, torch.floa
 
 def make_config(hidden_size: int, intermediate_size: int, num_local_experts: int, num_experts_per_tok: int,
                 swiglu_limit: float = 7.0, swiglu_alpha: float = 1.702, dtype: str = "bf16",
-                wfmt: str = "dense", y_f32: bool = False) -> MoeConfig:
-    """y_f32: the layer output y is stored in fp32 (the sums before their rounding to dtype)."""
+                wfmt: str = "dense", y_f32: bool = False, h_split: bool = False) -> MoeConfig:
+    """y_f32: the layer output y is stored in fp32 (the sums before their rounding to dtype).
+    h_split: the SwiGLU output is kept as two bf16 halves (hi + lo) between the expert GEMMs."""
     return MoeConfig(hidden_size, intermediate_size, num_local_experts, num_experts_per_tok, swiglu_limit,
                      swiglu_alpha, _DT[dtype][0], _lib.MOE_W_MXFP4 if wfmt == "mxfp4" else _lib.MOE_W_DENSE,
-                     1 if y_f32 else 0)
+                     1 if y_f32 else 0, 1 if h_split else 0)
 
 
-def config_from_spec(spec, y_f32: bool = False) -> MoeConfig:
+def config_from_spec(spec, y_f32: bool = False, h_split: bool = False) -> MoeConfig:
     """Config of a ``workloads.LayerSpec``."""
-    return make_config(spec.D, spec.F, spec.E, spec.k, spec.limit, spec.alpha, spec.dtype, spec.wfmt, y_f32)
+    return make_config(spec.D, spec.F, spec.E, spec.k, spec.limit, spec.alpha, spec.dtype, spec.wfmt, y_f32,
+                       h_split)
 
 
 def torch_dtype(cfg: MoeConfig) -> torch.dtype:
@@ -265,7 +267,9 @@ def expert_ffn(cfg: MoeConfig, x_perm: torch.Tensor, expert_off: torch.Tensor, w
     L = _lib.load()
     R, dev = x_perm.shape[0], x_perm.device
     dt = torch_dtype(cfg)
-    h = torch.empty((R, cfg.intermediate_size), dtype=dt, device=dev)
+    # with h_split (bf16) each row of h holds the bf16 halves hi and lo: [R, 2, F]
+    halves = 2 if (cfg.h_split and cfg.dtype == _lib.MOE_BF16) else 1
+    h = torch.empty((R, halves * cfg.intermediate_size), dtype=dt, device=dev)
     y_perm = torch.empty((R, cfg.hidden_size), dtype=dt, device=dev)
     nws = _size(L.moe_expert_ffn_workspace_size(ctypes.byref(cfg), T), "moe_expert_ffn_workspace_size")
     ws = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
@@ -347,9 +351,9 @@ def glm_expert_weights_from(d: Dict[str, torch.Tensor]) -> ExpertWeights:
     return ExpertWeights(d["w_gate"], d["w_up"], d["w_down"], None, None, None)
 
 
-def glm_config_from_spec(spec, y_f32: bool = False) -> MoeConfig:
+def glm_config_from_spec(spec, y_f32: bool = False, h_split: bool = False) -> MoeConfig:
     """Config of a ``workloads.GlmLayerSpec`` (the SwiGLU limit and alpha are not used by the variant)."""
-    return make_config(spec.D, spec.F, spec.E, spec.k, dtype=spec.dtype, y_f32=y_f32)
+    return make_config(spec.D, spec.F, spec.E, spec.k, dtype=spec.dtype, y_f32=y_f32, h_split=h_split)
 
 
 def check_glm_args(cfg: MoeConfig, params: GlmParams, x, w_router, weights: Optional[ExpertWeights] = None,

@@ -107,7 +107,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int G = args.num_groups;
   const int FB = (args.n_out + FBW - 1) / FBW;
   const int KB = (args.k_dim + BK - 1) / BK;
-  const int KSTEP_STAGES = (KB + KBS - 1) / KBS;      // stages per unit (blocks past K read zeros)
+  // down over h kept as two bf16 halves: K blocks [0, KB) read hi, [KB, 2 KB) lo (same weights)
+  const bool hsplit = !kGateUp && args.h_halves == 2;
+  const int KBT = hsplit ? 2 * KB : KB;
+  const int KSTEP_STAGES = (KBT + KBS - 1) / KBS;     // stages per unit (blocks past K read zeros)
   const uint64_t lim = args.wait_limit_ns;
 
   if (threadIdx.x == 0) {
@@ -202,10 +205,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (kGateUp) {
               tma_load_3d(sw, &tmW0, &full[s], kb * BK, ui.f0, ui.g);
               tma_load_3d(sw + 64 * kRowBytes, &tmW1, &full[s], kb * BK, ui.f0, ui.g);
+              tma_load_2d(sx, &tmX, &full[s], kb * BK, ui.m0);
+            } else if (hsplit) {
+              // blocks past 2 KB fall outside both the halves and the weights: zeros
+              const int half = kb / KB;
+              const int kbl = kb - half * KB;
+              tma_load_3d(sw, &tmW0, &full[s], kbl * BK, ui.f0, ui.g);
+              tma_load_3d(sx, &tmX, &full[s], kbl * BK, half, ui.m0);
             } else {
               tma_load_3d(sw, &tmW0, &full[s], kb * BK, ui.f0, ui.g);
+              tma_load_2d(sx, &tmX, &full[s], kb * BK, ui.m0);
             }
-            tma_load_2d(sx, &tmX, &full[s], kb * BK, ui.m0);
           }
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
@@ -308,7 +318,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const float gc = fminf(fmaxf(v[c] + bg, args.gate_lo), args.limit);
               const float uc = fminf(fmaxf(up_stage[wrow * NTOK + c] + bu, -args.limit), args.limit);
               const float h = __fdividef(gc * uc, 1.0f + __expf(-args.alpha * gc));
-              out[static_cast<size_t>(ui.m0 + c) * args.ldo + f] = __float2bfloat16_rn(h);
+              const T hi = __float2bfloat16_rn(h);
+              out[static_cast<size_t>(ui.m0 + c) * args.ldo + f] = hi;
+              if (args.h_halves == 2)
+                out[static_cast<size_t>(ui.m0 + c) * args.ldo + args.n_out + f] =
+                    __float2bfloat16_rn(h - __bfloat162float(hi));
             }
           }
           mbar_arrive(upempty);

@@ -55,6 +55,22 @@ static cudaError_t make_tmap(CUtensorMap* m, const void* ptr, bool f32, uint64_t
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// h kept as two bf16 halves per row, [rows][2][K]: dims {K, 2, rows}; a box is box_rows rows
+// of one half x 128 bytes, laid out in shared memory exactly as a [box_rows x 128 B] box of a
+// plain [rows, K] map (the middle dimension's box is 1).
+static cudaError_t make_tmap_halves(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {K, 2, rows};
+  const cuuint64_t strides[2] = {K * 2, K * 2 * 2};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kRowBytes / 2), 1, box_rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // Packed MXFP4 rows: [groups, rows, K/2] bytes, boxes of box_rows x 32 bytes (64 codes), no swizzle.
 static cudaError_t make_tmap_packed(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows, uint64_t groups,
                                    uint32_t box_rows) {
@@ -386,8 +402,9 @@ cudaError_t expert_down_mxfp4(const Launch& L, int64_t R, int D, int F, int E, c
 
 cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,
                           const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h,
-                          float gate_lo) {
+                          float gate_lo, int h_halves) {
   if (R == 0) return cudaSuccess;
+  if (h_halves == 2 && (!bf16 || gemm_kind(R, E) == GK_WM_PAIR)) return cudaErrorNotSupported;
   if (!bf16) {
     GemmArgs a = base_args(L);
     a.group_off = expert_off;
@@ -425,7 +442,8 @@ cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, i
   a.alpha = alpha;
   a.gate_lo = gate_lo;
   a.out = h;
-  a.ldo = F;
+  a.ldo = h_halves == 2 ? 2 * F : F;
+  a.h_halves = h_halves;
   if (gemm_kind(R, E) == GK_DECODE) {
     CUtensorMap wg, wu, tx;
     if ((e = make_tmap(&wg, w.w_gate, false, D, F, E, 64)) != cudaSuccess) return e;
@@ -456,8 +474,10 @@ cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, i
 
 cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* h,
                         const int32_t* expert_off, const ExpertWeights& w, const int32_t* slot_of_row,
-                        const float* topk_w, void* out) {
+                        const float* topk_w, void* out, int h_halves) {
   if (R == 0) return cudaSuccess;
+  const bool hsplit = h_halves == 2;
+  if (hsplit && (!bf16 || gemm_kind(R, E, true) == GK_WM_PAIR)) return cudaErrorNotSupported;
   if (!bf16) {
     GemmArgs a = base_args(L);
     a.group_off = expert_off;
@@ -482,7 +502,9 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
   }
   CUtensorMap ta, tb;
   cudaError_t e;
-  if ((e = make_tmap(&ta, h, !bf16, F, R, 0, kBM)) != cudaSuccess) return e;
+  if (hsplit) e = make_tmap_halves(&ta, h, F, R, kBM);
+  else e = make_tmap(&ta, h, !bf16, F, R, 0, kBM);
+  if (e != cudaSuccess) return e;
   GemmArgs a = base_args(L);
   a.group_off = expert_off;
   a.num_groups = E;
@@ -494,10 +516,13 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
   a.ldo = D;
   a.slot_of_row = slot_of_row;
   a.topk_w = topk_w;
+  a.h_halves = h_halves;
   if (gemm_kind(R, E, true) == GK_DECODE) {
     CUtensorMap wd, th;
     if ((e = make_tmap(&wd, w.w_down, false, F, D, E, 128)) != cudaSuccess) return e;
-    if ((e = make_tmap(&th, h, false, F, R, 0, kDecTok)) != cudaSuccess) return e;
+    if (hsplit) e = make_tmap_halves(&th, h, F, R, kDecTok);
+    else e = make_tmap(&th, h, false, F, R, 0, kDecTok);
+    if (e != cudaSuccess) return e;
     const int64_t units = (std::min<int64_t>(E, R) + R / kDecTok) * ((D + 127) / 128);
     if (slot_of_row != nullptr) {
       // the split needs a K stage (kDecKBS 64-wide K blocks) in each half: with a single

@@ -70,6 +70,10 @@ struct GemmArgs {
   const uint8_t* scale1;
   int k_splits;                // EPI_PARTIAL: K ranges; column block index = K range
   float* partial;              // EPI_PARTIAL: [k_splits, n_out, m_total] fp32
+  int h_halves;                // 2: h is kept as two bf16 halves per row, [R, 2, F] (h = hi + lo):
+                               // EPI_SWIGLU writes hi = bf16(h) and lo = bf16(h - hi); the down
+                               // GEMM reads h through a 3-D tensor map {F, 2, R} and sums over
+                               // both halves against the same weights (K = 2F).  0 or 1: one bf16 h.
 };
 
 constexpr int kBM = 128;           // rows per tile (MMA M)
@@ -146,6 +150,15 @@ __device__ __forceinline__ void epi_swiglu(uint32_t tbase, int row, bool rvalid,
         h[j] = __fdividef(gc * uc, 1.0f + __expf(-alpha * gc));
       }
       store8<T>(out + c, h);
+      if constexpr (!std::is_same<T, float>::value) {
+        if (a.h_halves == 2) {
+          // the part of h that its bf16 rounding dropped, itself in bf16 (h - hi is exact in fp32)
+          float lo[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) lo[j] = h[j] - __bfloat162float(__float2bfloat16_rn(h[j]));
+          store8<T>(out + a.n_out + c, lo);
+        }
+      }
     }
   }
 }
@@ -288,6 +301,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int NT = (EPI == EPI_PARTIAL) ? args.k_splits : (args.n_out + TN - 1) / TN;
   const int KB = (args.k_dim + BK - 1) / BK;
   const int KBS = (EPI == EPI_PARTIAL) ? (KB + args.k_splits - 1) / args.k_splits : KB;   // k-blocks per range
+  // down projection over h kept as two bf16 halves: K blocks [0, KB) read hi, [KB, 2 KB) lo,
+  // both against the weights' K blocks [0, KB)
+  const bool hsplit = (EPI == EPI_BIAS || EPI == EPI_BIAS_WSCATTER) && args.h_halves == 2;
+  const int KBT = hsplit ? 2 * KB : KB;
   const uint64_t lim = args.wait_limit_ns;
   // k-block range of a tile: all of K, or (EPI_PARTIAL) the range of its column block index
   auto kb_range = [&](const TileInfo& ti, int& b, int& e) {
@@ -297,7 +314,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       e = min(KB, b + KBS);
     } else {
       b = 0;
-      e = KB;
+      e = KBT;
     }
   };
 
@@ -378,8 +395,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(&full[s], tx_bytes);
           uint8_t* sa = smem + s * LY::STAGE_BYTES;
           uint8_t* sb = sa + LY::A_BYTES;
-          tma_load_2d(sa, &tmA, &full[s], kb * BK, ti.m0);
-          tma_load_3d(sb, &tmB0, &full[s], kb * BK, b_row, ti.g);
+          const int half = hsplit ? kb / KB : 0;
+          const int kbl = kb - half * KB;
+          if (hsplit) tma_load_3d(sa, &tmA, &full[s], kbl * BK, half, ti.m0);
+          else tma_load_2d(sa, &tmA, &full[s], kb * BK, ti.m0);
+          tma_load_3d(sb, &tmB0, &full[s], kbl * BK, b_row, ti.g);
           if (NB == 2) tma_load_3d(sb + TN * kRowBytes, &tmB1, &full[s], kb * BK, ti.n0, ti.g);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);

@@ -97,6 +97,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int G = args.num_groups;
   const int NT = (args.n_out + TNO - 1) / TNO;
   const int KB = (args.k_dim + BK - 1) / BK;
+  // down over h kept as two bf16 halves: K blocks [0, KB) read hi, [KB, 2 KB) lo (same weights)
+  const bool hsplit = EPI != EPI_SWIGLU && args.h_halves == 2;
+  const int KBT = hsplit ? 2 * KB : KB;
   const uint64_t lim = args.wait_limit_ns;
 
   if (threadIdx.x == 0) {
@@ -171,14 +174,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const TileInfo ti = decode_pair_tile(i, tile_off, goff, G, NT, TNO);
         const int a_row = ti.m0 + static_cast<int>(rank) * 128;
         const int b_row = (EPI == EPI_SWIGLU) ? ti.n0 : ti.n0 + static_cast<int>(rank) * TNH;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = 0; kb < KBT; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) { ok = false; break; }
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * LY::STAGE_BYTES);
           uint8_t* sa = smem + s * LY::STAGE_BYTES;
           uint8_t* sb = sa + LY::A_BYTES;
           const uint32_t fb = full_leader + static_cast<uint32_t>(s) * 8u;
-          tma_load_2d_pair(sa, &tmA, fb, kb * BK, a_row);
-          tma_load_3d_pair(sb, tmb, fb, kb * BK, b_row, ti.g);
+          const int half = hsplit ? kb / KB : 0;
+          const int kbl = kb - half * KB;
+          if (hsplit) tma_load_3d_pair(sa, &tmA, fb, kbl * BK, half, a_row);
+          else tma_load_2d_pair(sa, &tmA, fb, kb * BK, a_row);
+          tma_load_3d_pair(sb, tmb, fb, kbl * BK, b_row, ti.g);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -211,7 +217,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait_cluster(&tempty[acc], aph ^ 1u, abort_flag, lim)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = 0; kb < KBT; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag, lim)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * LY::STAGE_BYTES);

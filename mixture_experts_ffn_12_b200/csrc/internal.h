@@ -44,16 +44,19 @@ struct ExpertWeights {
 
 // h[R, F] = swiglu(x_perm W_g^T + b_g, x_perm W_u^T + b_u), per expert segment.
 // gate_lo is the gate's lower clip: 0 for the clipped SwiGLU; -inf with limit = inf and
-// alpha = 1 gives SiLU(g) * u.
+// alpha = 1 gives SiLU(g) * u.  h_halves = 2 (bf16 only): h is [R, 2, F], the bf16 rounding
+// of h and the bf16 rounding of what that dropped (cudaErrorNotSupported for the fp32
+// kernels and the weights-in-M pair kernel).
 cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,
                           const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h,
-                          float gate_lo = 0.0f);
+                          float gate_lo = 0.0f, int h_halves = 1);
 
 // Down projection.  If slot_of_row == nullptr: out[r] = h[r] W_d^T + b_d (permuted order, dtype);
 // else out[slot_of_row[r]] = topk_w[slot] * (h[r] W_d^T + b_d) (slot order, fp32).
+// h_halves = 2: h is [R, 2, F] as written by expert_gateup, and both halves are summed.
 cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* h,
                         const int32_t* expert_off, const ExpertWeights& w, const int32_t* slot_of_row,
-                        const float* topk_w, void* out);
+                        const float* topk_w, void* out, int h_halves = 1);
 
 // y[t] = sum_j w[t,j] * y_perm[row_of_slot[t,j]]   (y_perm in dtype; y in dtype, or fp32 if out_f32)
 cudaError_t combine_gather(const Launch& L, bool bf16, bool out_f32, int64_t T, int D, int k, const void* y_perm,

@@ -51,8 +51,18 @@ moe_status_t check_cfg(const moe_config_t* c) {
   if (!std::isfinite(c->swiglu_limit) || !(c->swiglu_limit > 0.0f) || !std::isfinite(c->swiglu_alpha))
     return MOE_ERR_INVALID_ARG;
   if (c->y_f32 != 0 && c->y_f32 != 1) return MOE_ERR_INVALID_ARG;
+  if (c->h_split != 0 && c->h_split != 1) return MOE_ERR_INVALID_ARG;
   if (c->wfmt == MOE_W_MXFP4 && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (c->wfmt == MOE_W_MXFP4 && c->h_split != 0) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
+}
+
+// h kept as two bf16 halves (bf16 layers; fp32 layers keep h in fp32 and ignore the flag)
+int h_halves(const moe_config_t* c) { return (c->dtype == MOE_BF16 && c->h_split != 0) ? 2 : 1; }
+
+// checked before any launch: the weights-in-M pair kernels have no two-halves form
+moe_status_t check_variant(const moe_config_t* c) {
+  return (h_halves(c) == 2 && moe::g_gemm_variant.load() == 4) ? MOE_ERR_UNSUPPORTED : MOE_OK;
 }
 
 // the layer output is bf16 only for a bf16 layer without y_f32
@@ -101,7 +111,7 @@ Layout layout(const moe_config_t* c, int64_t T) {
   L.xperm = take(R * c->hidden_size * (es > 4 ? es : 4));
   L.ys = L.xperm;
   // the router's K-split partial logits are dead before gate/up writes h: they share it
-  const size_t h_bytes = R * c->intermediate_size * es;
+  const size_t h_bytes = R * c->intermediate_size * es * h_halves(c);
   const size_t rpart_bytes = moe::router_partial_bytes(T, c->num_local_experts);
   L.h = take(h_bytes > rpart_bytes ? h_bytes : rpart_bytes);
   L.rpart = L.h;
@@ -179,11 +189,14 @@ moe_status_t run_experts(const moe_config_t* c, const Launch& L, int64_t T, cons
     stage_mark(ST_DOWN, false, L.stream);
     return st;
   }
-  if (moe::expert_gateup(L, bf16, R, D, F, E, x_perm, eoff, w, c->swiglu_limit, c->swiglu_alpha, h) != cudaSuccess)
+  const int hh = h_halves(c);
+  if (moe::expert_gateup(L, bf16, R, D, F, E, x_perm, eoff, w, c->swiglu_limit, c->swiglu_alpha, h, 0.0f, hh) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   stage_mark(ST_GATEUP, false, L.stream);
   stage_mark(ST_DOWN, true, L.stream);
-  const moe_status_t st = cuda_status(moe::expert_down(L, bf16, R, D, F, E, h, eoff, w, slot_of_row, topk_w, out));
+  const moe_status_t st =
+      cuda_status(moe::expert_down(L, bf16, R, D, F, E, h, eoff, w, slot_of_row, topk_w, out, hh));
   stage_mark(ST_DOWN, false, L.stream);
   return st;
 }
@@ -286,7 +299,7 @@ GlmLayout glm_layout(const moe_config_t* c, const moe_glm_params_t* p, int64_t T
   L.pscr = take(moe::permute_scratch_words(T, c->num_local_experts) * 4);
   L.xperm = take(R * D * (es > 4 ? es : 4));   // x_perm, then the weighted fp32 rows
   L.ys = L.xperm;
-  const size_t h_bytes = R * F * es, rpart_bytes = moe::router_partial_bytes(T, c->num_local_experts);
+  const size_t h_bytes = R * F * es * h_halves(c), rpart_bytes = moe::router_partial_bytes(T, c->num_local_experts);
   L.h = take(h_bytes > rpart_bytes ? h_bytes : rpart_bytes);
   L.rpart = L.h;
   // zero biases: [E, F] for gate/up, [E, D] for down, [1, Fs] / [1, D] for the shared expert
@@ -297,7 +310,7 @@ GlmLayout glm_layout(const moe_config_t* c, const moe_glm_params_t* p, int64_t T
     L.soff = take(2 * 4);
     L.sid = take(size_t(T) * 4);
     L.sone = take(size_t(T) * 4);
-    L.hs = take(size_t(T) * Fs * es);
+    L.hs = take(size_t(T) * Fs * es * h_halves(c));
     L.ysh = take(size_t(T) * D * 4);
   }
   L.total = o;
@@ -406,6 +419,7 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, int64_t T, const void* x_pe
   if (T == 0) return MOE_OK;
   if (!ptr_ok(x_perm) || !ptr_ok(expert_off) || !ptr_ok(h) || !ptr_ok(y_perm) || !weights_ok(cfg, weights))
     return MOE_ERR_INVALID_ARG;
+  if ((s = check_variant(cfg)) != MOE_OK) return s;
   const size_t need = ffn_ws_bytes(cfg, T);
   if (need > 0 && (ws == nullptr || !aligned16(ws) || ws_bytes < need)) return MOE_ERR_WORKSPACE;
   Launch L;
@@ -437,6 +451,7 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x
     return MOE_ERR_INVALID_ARG;
   if ((topk_ids_out != nullptr && !aligned16(topk_ids_out)) || (topk_w_out != nullptr && !aligned16(topk_w_out)))
     return MOE_ERR_INVALID_ARG;
+  if ((s = check_variant(cfg)) != MOE_OK) return s;
   const Layout LY = layout(cfg, T);
   if (ws == nullptr || !aligned16(ws) || ws_bytes < LY.total) return MOE_ERR_WORKSPACE;
   Launch L;
@@ -543,6 +558,7 @@ moe_status_t moe_glm_layer_forward(const moe_config_t* cfg, const moe_glm_params
   if (p->e_score_correction_bias != nullptr && !aligned16(p->e_score_correction_bias)) return MOE_ERR_INVALID_ARG;
   if ((topk_ids_out != nullptr && !aligned16(topk_ids_out)) || (topk_w_out != nullptr && !aligned16(topk_w_out)))
     return MOE_ERR_INVALID_ARG;
+  if ((s = check_variant(cfg)) != MOE_OK) return s;
   const GlmLayout LY = glm_layout(cfg, p, T);
   if (ws == nullptr || !aligned16(ws) || ws_bytes < LY.total) return MOE_ERR_WORKSPACE;
   Launch L;
@@ -583,9 +599,10 @@ moe_status_t moe_glm_layer_forward(const moe_config_t* cfg, const moe_glm_params
   rw.b_gate = zb;
   rw.b_up = zb;
   rw.b_down = zb;
-  if (moe::expert_gateup(L, bf16, R, D, F, E, xperm, eoff, rw, kInf, 1.0f, h, -kInf) != cudaSuccess)
+  const int hh = h_halves(cfg);
+  if (moe::expert_gateup(L, bf16, R, D, F, E, xperm, eoff, rw, kInf, 1.0f, h, -kInf, hh) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (moe::expert_down(L, bf16, R, D, F, E, h, eoff, rw, sor, w, ys) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::expert_down(L, bf16, R, D, F, E, h, eoff, rw, sor, w, ys, hh) != cudaSuccess) return MOE_ERR_CUDA;
   void* ysh = nullptr;
   if (Fs > 0) {
     int32_t* soff = reinterpret_cast<int32_t*>(base + LY.soff);
@@ -601,10 +618,11 @@ moe_status_t moe_glm_layer_forward(const moe_config_t* cfg, const moe_glm_params
     int32_t* sid = reinterpret_cast<int32_t*>(base + LY.sid);
     float* sone = reinterpret_cast<float*>(base + LY.sone);
     if (moe::glm_shared_off(L, T, soff, sid, sone) != cudaSuccess) return MOE_ERR_CUDA;
-    if (moe::expert_gateup(L, bf16, T, D, Fs, 1, x, soff, sw, kInf, 1.0f, hs, -kInf) != cudaSuccess)
+    if (moe::expert_gateup(L, bf16, T, D, Fs, 1, x, soff, sw, kInf, 1.0f, hs, -kInf, hh) != cudaSuccess)
       return MOE_ERR_CUDA;
     // fp32 rows (identity slots, unit weights): the shared output is rounded once, with the sum
-    if (moe::expert_down(L, bf16, T, D, Fs, 1, hs, soff, sw, sid, sone, ysh) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe::expert_down(L, bf16, T, D, Fs, 1, hs, soff, sw, sid, sone, ysh, hh) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   return cuda_status(moe::combine_slots_shared(L, out_bf16(cfg), T, D, k, ys, ysh, y));
 }

@@ -80,6 +80,50 @@ def check_rounding(y_out, y32, ref: np.ndarray = None) -> None:
               f"exact result rounded to bf16: {np.max(np.abs(exact_rounded - ref)) / rms:.3e}")
 
 
+def h_rounding_bound(layer, ids: np.ndarray, w: np.ndarray, h: np.ndarray) -> np.ndarray:
+    """Per-element bound on how far keeping h in bf16 can move the layer output.
+
+    Each stored h value differs from the exact one by its bf16 rounding, at most
+    2^-9 |h| (plus a little fp32 arithmetic), so |delta y[t, d]| <=
+    2^-9 * sum_j w[t, j] * sum_f |h[t, j, f]| |W_d[e_j][d, f]|.  Returned with the
+    factor 2^-8 (twice the rounding bound) as margin for the fp32 side.
+    ids, w [n, k] and h [n, k, F] are the oracle's, for the n tokens compared.
+    """
+    n, k = ids.shape
+    out = np.zeros((n, layer["b_down"].shape[1]))
+    for e in np.unique(ids):
+        ii, jj = np.nonzero(ids == e)
+        wd = np.abs(O.expert_weights(layer, "down", int(e)))
+        out[ii] += w[ii, jj][:, None] * (np.abs(h[ii, jj]) @ wd.T)
+    return 2.0 ** -8 * out
+
+
+def h_rounding_bound_glm(layer, ref) -> np.ndarray:
+    """h_rounding_bound for the GLM4-MoE-Lite variant: the routed experts' h (oracle, permuted
+    order) and the shared expert's h, each against |W_d| of its expert."""
+    from oracle import glm_moe as G
+    ids, w, ros, h = ref["ids"], ref["w"], ref["row_of_slot"], ref["h"]
+    T, k = ids.shape
+    out = np.zeros((T, layer["w_down"].shape[1]))
+    for e in np.unique(ids):
+        ii, jj = np.nonzero(ids == e)
+        wd = np.abs(G.decode(layer["w_down"][int(e)]))
+        out[ii] += w[ii, jj][:, None] * (np.abs(h[ros[ii, jj]]) @ wd.T)
+    if "ws_gate" in layer:
+        x = G.decode(layer["x"])
+        hs, _ = G.silu_mlp(x, G.decode(layer["ws_gate"]), G.decode(layer["ws_up"]), G.decode(layer["ws_down"]))
+        out += np.abs(hs) @ np.abs(G.decode(layer["ws_down"])).T
+    return 2.0 ** -8 * out
+
+
+def check_h_rounding(y_default: np.ndarray, y_split: np.ndarray, bound: np.ndarray, ref: np.ndarray) -> None:
+    """The layer with h in one bf16 value differs from the layer with h in two bf16 halves
+    by no more than the bf16 rounding of h can explain (both outputs in fp32)."""
+    rms = float(np.sqrt(np.mean(np.square(ref))))
+    excess = np.abs(y_default - y_split) - (bound + 1e-4 * rms)
+    assert np.all(excess <= 0), f"h-in-bf16 output off by more than its rounding: excess {excess.max():.3e}"
+
+
 def rel_rms(got: np.ndarray, ref: np.ndarray) -> float:
     rms = float(np.sqrt(np.mean(np.square(ref))))
     return float(np.max(np.abs(got - ref))) / max(rms, 1e-30)

@@ -32,8 +32,9 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_struct_layout_matches_header():
-    assert ctypes.sizeof(_lib.MoeConfig) == 36
+    assert ctypes.sizeof(_lib.MoeConfig) == 40
     assert _lib.MoeConfig.y_f32.offset == 32
+    assert _lib.MoeConfig.h_split.offset == 36
     assert ctypes.sizeof(_lib.MoeExpertWeights) == 9 * ctypes.sizeof(ctypes.c_void_p)
     # int32, float, four pointers, int32 (+ tail padding to pointer alignment)
     assert ctypes.sizeof(_lib.MoeGlmParams) == 48
@@ -77,6 +78,10 @@ def test_version_and_status_strings(lib):
     (dict(y_f32=1, dtype=_lib.MOE_F32), _lib.MOE_OK),
     (dict(y_f32=2), _lib.MOE_ERR_INVALID_ARG),
     (dict(y_f32=-1), _lib.MOE_ERR_INVALID_ARG),
+    (dict(h_split=1), _lib.MOE_OK),
+    (dict(h_split=1, dtype=_lib.MOE_F32), _lib.MOE_OK),          # fp32 layers keep h in fp32 anyway
+    (dict(h_split=1, wfmt=_lib.MOE_W_MXFP4), _lib.MOE_ERR_UNSUPPORTED),
+    (dict(h_split=3), _lib.MOE_ERR_INVALID_ARG),
 ])
 def test_config_check(lib, kw, want):
     assert lib.moe_config_check(ctypes.byref(cfg(**kw))) == want
@@ -138,6 +143,26 @@ def test_rejections_launch_nothing(lib):
         _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_layer_forward(ctypes.byref(c), 0, None, None, None, None, None, None, None, None, 0, None) == \
         _lib.MOE_OK
+
+
+def test_h_split_workspace_and_variant_check(lib):
+    """h in two bf16 halves doubles the h region of the workspace; the weights-in-M pair
+    kernels have no such form, and the call says so before launching anything."""
+    T, k, F = 4096, 4, 2880
+    c, cs = cfg(), cfg(h_split=1)
+    assert lib.moe_workspace_size(ctypes.byref(cs), T) - lib.moe_workspace_size(ctypes.byref(c), T) == T * k * F * 2
+    c32, c32s = cfg(dtype=_lib.MOE_F32), cfg(dtype=_lib.MOE_F32, h_split=1)
+    assert lib.moe_workspace_size(ctypes.byref(c32), T) == lib.moe_workspace_size(ctypes.byref(c32s), T)
+    p = ctypes.c_void_p(0x10000)
+    w = _lib.MoeExpertWeights(*([0x10000] * 3 + [None] * 3 + [0x10000] * 3))
+    assert lib.moe_set_expert_gemm_variant(4) == _lib.MOE_OK
+    try:
+        assert lib.moe_layer_forward(ctypes.byref(cs), 8, p, p, p, ctypes.byref(w), p, None, None, p, 1 << 40,
+                                     None) == _lib.MOE_ERR_UNSUPPORTED
+        assert lib.moe_expert_ffn(ctypes.byref(cs), 8, p, p, ctypes.byref(w), p, p, None, 0, None) == \
+            _lib.MOE_ERR_UNSUPPORTED
+    finally:
+        assert lib.moe_set_expert_gemm_variant(0) == _lib.MOE_OK
 
 
 def glm_params(**kw):

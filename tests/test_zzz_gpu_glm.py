@@ -3,16 +3,19 @@
 Source of the variant: "Ollama glm4_moe_lite.go" (MoEGate.Forward, SwitchMLP.Forward,
 SharedExperts.Forward, MoE.Forward).  Bit-exact: the chosen expert sets (and their
 order where the corrected scores are separated).  Routing weights within 2e-5 (they
-include routed_scaling_factor).  Each layer call runs with the output in the layer
-dtype and in fp32 (y_f32): the fp32 output within 2e-2 of the output's RMS, the
-bound of the GPT-OSS layer as written, and the dtype output exactly its rounding.
+include routed_scaling_factor).  Each layer runs with the output in the layer dtype
+and in fp32 (y_f32), and (bf16) with h kept as two bf16 halves (h_split): that
+form's fp32 output within 2e-2 of the output's RMS, the bound of the GPT-OSS layer
+as written; the default form within the bf16 rounding of h of it; the dtype output
+exactly the rounding of the fp32 output.
 """
 import numpy as np
 import pytest
 
 import workloads as W
 from oracle import glm_moe as G
-from parity_util import TOL_W, TOL_Y, check_ids, check_output, check_rounding, f64
+from parity_util import (TOL_W, TOL_Y, check_h_rounding, check_ids, check_output, check_rounding, f64,
+                         h_rounding_bound_glm)
 
 pytestmark = pytest.mark.gpu
 
@@ -48,13 +51,15 @@ def _layer(spec):
     return W.make_glm_layer(spec, seed=0, scores_fn=_scores_fn(spec))
 
 
-def _run(api, spec, layer):
-    """The layer with y in its dtype and with y in fp32: (y, y32, ids, w)."""
+def _run(api, spec, layer, split=True):
+    """The layer with y in its dtype, with y in fp32, and (bf16, `split`) with y in fp32 and h
+    in two bf16 halves: (y, y32, y32s or None, ids, w)."""
     d = api.upload_layer(layer)
     params = api.glm_params_from(spec, d)
     out = []
-    for y_f32 in (False, True):
-        cfg = api.glm_config_from_spec(spec, y_f32=y_f32)
+    modes = [(False, False), (True, False)] + ([(True, True)] if split and spec.dtype == "bf16" else [])
+    for y_f32, h_split in modes:
+        cfg = api.glm_config_from_spec(spec, y_f32=y_f32, h_split=h_split)
         ids = torch.empty((spec.T, spec.k), dtype=torch.int32, device="cuda")
         w = torch.empty((spec.T, spec.k), dtype=torch.float32, device="cuda")
         y = api.glm_layer_forward(cfg, params, d["x"], d["w_router"], api.glm_expert_weights_from(d),
@@ -62,14 +67,23 @@ def _run(api, spec, layer):
         torch.cuda.synchronize()
         assert api.last_device_error() == 0
         out.append((y, ids, w))
-    (y, ids, w), (y32, ids32, w32) = out
-    assert torch.equal(ids, ids32) and torch.equal(w, w32)
-    return y, y32, ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+    y, ids, w = out[0]
+    for _, ids2, w2 in out[1:]:
+        assert torch.equal(ids, ids2) and torch.equal(w, w2)
+    y32s = out[2][0] if len(out) > 2 else None
+    return y, out[1][0], y32s, ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
 
 
-def _check_layer(y, y32, ref_y, tol):
-    check_output(f64(y32), ref_y, tol)
-    check_rounding(y, y32, ref_y)
+def _check_layer(y, y32, y32s, ref, tol, layer):
+    if y32s is not None:
+        print("h in two bf16 halves:", end=" ")
+        check_output(f64(y32s), ref["y"], tol)
+        check_h_rounding(f64(y32), f64(y32s), h_rounding_bound_glm(layer, ref), ref["y"])
+        rms = float(np.sqrt(np.mean(np.square(ref["y"]))))
+        print(f"h in bf16: max err / RMS = {np.max(np.abs(f64(y32) - ref['y'])) / rms:.3e}")
+    else:
+        check_output(f64(y32), ref["y"], tol)
+    check_rounding(y, y32, ref["y"])
 
 
 def _check_weights(gid, gw, rid, rw):
@@ -81,11 +95,11 @@ def _check_weights(gid, gw, rid, rw):
 @pytest.mark.parametrize("spec", SPECS, ids=lambda s: s.name)
 def test_glm_layer_forward(api, spec):
     layer = _layer(spec)
-    y, y32, gid, gw = _run(api, spec, layer)
+    y, y32, y32s, gid, gw = _run(api, spec, layer)
     ref = G.layer_forward(layer, spec.k, spec.norm_topk_prob, spec.routed_scaling_factor)
     check_ids(gid, ref["ids"], ref["chosen_by"])
     _check_weights(gid, gw, ref["ids"], ref["w"])
-    _check_layer(y, y32, ref["y"], TOL_Y[spec.dtype])
+    _check_layer(y, y32, y32s, ref, TOL_Y[spec.dtype], layer)
 
 
 @pytest.mark.parametrize("spec", [GLM_TC_ROUTER, GLM_F32, GLM_K1, GLM_MANY], ids=lambda s: s.name)
@@ -112,12 +126,12 @@ def test_glm_each_gemm_variant(api, variant):
     layer = _layer(spec)
     api.set_expert_gemm_variant(variant)
     try:
-        y, y32, gid, _ = _run(api, spec, layer)
+        y, y32, y32s, gid, _ = _run(api, spec, layer, split=variant != 4)
     finally:
         api.set_expert_gemm_variant(0)
     ref = G.layer_forward(layer, spec.k, spec.norm_topk_prob, spec.routed_scaling_factor)
     check_ids(gid, ref["ids"], ref["chosen_by"])
-    _check_layer(y, y32, ref["y"], TOL_Y["bf16"])
+    _check_layer(y, y32, y32s, ref, TOL_Y["bf16"], layer)
 
 
 def test_glm_zero_tokens(api):
