@@ -80,7 +80,17 @@ typedef enum {
 } moe_status_t;
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
-typedef enum { MOE_W_DENSE = 0, MOE_W_MXFP4 = 1 } moe_wfmt_t;
+/* MOE_W_MXFP4_A8: the MXFP4 weights of MOE_W_MXFP4, multiplied on the
+ * block-scaled tensor cores (tcgen05.mma kind::mxf8f6f4) with the activations of
+ * both expert projections (x_perm and h) quantized to MXFP8: E4M3 elements, one
+ * E8M0 scale per 32 elements along K, the scale 2^X the smallest power of two
+ * with the block's largest magnitude <= 448 * 2^X (no element saturates),
+ * elements rounded to nearest, ties to even.  A numerics variant of the layer
+ * (the pages name MXFP8 and its group size 32, "Ollama glm4_moe_lite.go",
+ * quantizationParams); its results differ from MOE_W_MXFP4 by that
+ * quantization.  Needs D and F multiples of 64 and weight pointers 32-byte
+ * aligned; moe_layer_forward only (moe_expert_ffn returns MOE_ERR_UNSUPPORTED). */
+typedef enum { MOE_W_DENSE = 0, MOE_W_MXFP4 = 1, MOE_W_MXFP4_A8 = 2 } moe_wfmt_t;
 
 /* Field names follow the GPT-OSS Config (hidden_size, num_local_experts,
  * num_experts_per_tok, swiglu_limit); intermediate_size is F. */
@@ -227,6 +237,20 @@ MOE_API moe_status_t moe_combine(const moe_config_t* cfg, int64_t T, const void*
 MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x, const void* w_router,
                                const void* b_router, const moe_expert_weights_t* weights, void* y,
                                int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
+
+/* MXFP8 quantization of activation rows, the one MOE_W_MXFP4_A8 applies to x_perm
+ * and h (the pages give MXFP8 and its group size 32, "Ollama glm4_moe_lite.go",
+ * quantizationParams; the scale rule and rounding are this library's reading):
+ *   x [rows, K] bf16 (K a multiple of 32)
+ *   -> xq [rows, K] uint8 E4M3 codes (sign bit 7, exponent bits 6..3 bias 7,
+ *        mantissa bits 2..0), xq[r, j] = RNE(x[r, j] / 2^X) for j in block b,
+ *      sf [rows, moe_mxfp8_scale_stride(K)] uint8: sf[r, b] = X + 127 for the
+ *        K/32 blocks b, X the smallest integer with max |x| of the block <=
+ *        448 * 2^X (-127 for an all-zero block), then 127 up to the stride.
+ * Device pointers, 16-byte aligned.  rows = 0 is a no-op. */
+MOE_API int32_t moe_mxfp8_scale_stride(int32_t K);
+MOE_API moe_status_t moe_quantize_mxfp8(int64_t rows, int32_t K, const void* x, uint8_t* xq, uint8_t* sf,
+                                        void* stream);
 
 /* Reads and clears the current device's error word (synchronises the device).
  * MOE_OK if no kernel flagged anything since the last call, MOE_ERR_TIMEOUT if a

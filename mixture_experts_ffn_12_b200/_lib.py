@@ -18,7 +18,7 @@ MOE_ERR_TIMEOUT = 5
 MOE_ERR_DEVICE_BOUNDS = 6
 
 MOE_F32, MOE_BF16 = 0, 1
-MOE_W_DENSE, MOE_W_MXFP4 = 0, 1
+MOE_W_DENSE, MOE_W_MXFP4, MOE_W_MXFP4_A8 = 0, 1, 2
 
 SIZE_INVALID = ctypes.c_size_t(-1).value
 ABI_VERSION = 2
@@ -76,6 +76,8 @@ SIGNATURES = {
     "moe_expert_ffn": (_ST, [_CFG, _I64, _P, _P, _W, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_combine": (_ST, [_CFG, _I64, _P, _P, _P, _P, _P]),
     "moe_layer_forward": (_ST, [_CFG, _I64, _P, _P, _P, _W, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_mxfp8_scale_stride": (ctypes.c_int32, [ctypes.c_int32]),
+    "moe_quantize_mxfp8": (_ST, [_I64, ctypes.c_int32, _P, _P, _P, _P]),
     "moe_last_device_error": (_ST, []),
     "moe_set_stage_events": (None, [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p),
                                     ctypes.c_int32]),

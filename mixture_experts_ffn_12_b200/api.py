@@ -31,6 +31,9 @@ def _check(code: int, what: str) -> None:
 
 
 _DT = {"bf16": (_lib.MOE_BF16, torch.bfloat16), "f32": (_lib.MOE_F32, torch.float32)}
+# expert-weight formats: dense, MXFP4 (decoded to bf16 in the GEMM mainloop), MXFP4 with MXFP8
+# activations on the block-scaled tensor cores
+_WF = {"dense": _lib.MOE_W_DENSE, "mxfp4": _lib.MOE_W_MXFP4, "mxfp4_a8": _lib.MOE_W_MXFP4_A8}
 
 
 def make_config(hidden_size: int, intermediate_size: int, num_local_experts: int, num_experts_per_tok: int,
@@ -39,14 +42,14 @@ def make_config(hidden_size: int, intermediate_size: int, num_local_experts: int
     """y_f32: the layer output y is stored in fp32 (the sums before their rounding to dtype).
     h_split: the SwiGLU output is kept as two bf16 halves (hi + lo) between the expert GEMMs."""
     return MoeConfig(hidden_size, intermediate_size, num_local_experts, num_experts_per_tok, swiglu_limit,
-                     swiglu_alpha, _DT[dtype][0], _lib.MOE_W_MXFP4 if wfmt == "mxfp4" else _lib.MOE_W_DENSE,
-                     1 if y_f32 else 0, 1 if h_split else 0)
+                     swiglu_alpha, _DT[dtype][0], _WF[wfmt], 1 if y_f32 else 0, 1 if h_split else 0)
 
 
-def config_from_spec(spec, y_f32: bool = False, h_split: bool = False) -> MoeConfig:
-    """Config of a ``workloads.LayerSpec``."""
-    return make_config(spec.D, spec.F, spec.E, spec.k, spec.limit, spec.alpha, spec.dtype, spec.wfmt, y_f32,
-                       h_split)
+def config_from_spec(spec, y_f32: bool = False, h_split: bool = False, wfmt: Optional[str] = None) -> MoeConfig:
+    """Config of a ``workloads.LayerSpec``; `wfmt` overrides the spec's weight format (the MXFP4
+    weights of a spec also run as "mxfp4_a8")."""
+    return make_config(spec.D, spec.F, spec.E, spec.k, spec.limit, spec.alpha, spec.dtype, wfmt or spec.wfmt,
+                       y_f32, h_split)
 
 
 def torch_dtype(cfg: MoeConfig) -> torch.dtype:
@@ -102,7 +105,7 @@ def check_expert_weights(cfg: MoeConfig, w: "ExpertWeights", device: Optional[to
     [E, D, F/32], all uint8.  Biases [E, F], [E, F], [E, D] in the layer dtype."""
     D, F, E = cfg.hidden_size, cfg.intermediate_size, cfg.num_local_experts
     dt = torch_dtype(cfg)
-    if cfg.wfmt == _lib.MOE_W_MXFP4:
+    if cfg.wfmt in (_lib.MOE_W_MXFP4, _lib.MOE_W_MXFP4_A8):
         if D % 32 or F % 32:
             raise ValueError(f"MXFP4 weights need D and F divisible by 32 (D={D}, F={F})")
         _want("w_gate", w.w_gate, (E, F, D // 2), torch.uint8, device)
@@ -434,6 +437,20 @@ def glm_layer_forward(cfg: MoeConfig, params: GlmParams, x: torch.Tensor, w_rout
                                                  ws.numel() * ws.element_size(), _stream(dev)),
                "moe_glm_layer_forward")
     return y
+
+
+def quantize_mxfp8(x: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
+    """x [rows, K] bf16 -> (E4M3 codes [rows, K] uint8, E8M0 scale rows [rows, stride] uint8)."""
+    if x.dim() != 2 or x.dtype != torch.bfloat16:
+        raise ValueError("quantize_mxfp8 takes a 2-D bf16 tensor")
+    L = _lib.load()
+    rows, K = x.shape
+    stride = L.moe_mxfp8_scale_stride(K)
+    xq = torch.empty((rows, K), dtype=torch.uint8, device=x.device)
+    sf = torch.empty((rows, max(stride, 1)), dtype=torch.uint8, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(L.moe_quantize_mxfp8(rows, K, _p(x), _p(xq), _p(sf), _stream(x.device)), "moe_quantize_mxfp8")
+    return xq, sf
 
 
 def last_device_error() -> int:

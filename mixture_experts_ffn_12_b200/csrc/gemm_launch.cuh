@@ -15,6 +15,7 @@
 #include "decode_gemm.cuh"
 #include "grouped_gemm_pair.cuh"
 #include "grouped_gemm_pair_mx.cuh"
+#include "grouped_gemm_mx8.cuh"
 #include "grouped_gemm_wm_pair.cuh"
 #include "internal.h"
 #include "simt_gemm.cuh"
@@ -562,6 +563,161 @@ cudaError_t expert_down(const Launch& L, bool bf16, int64_t R, int D, int F, int
   if (slot_of_row != nullptr)
     return launch<__nv_bfloat16, kTNDown, 1, EPI_BIAS_WSCATTER, kStages>(L, ta, tb, tb, a, tiles);
   return launch<__nv_bfloat16, kTNDown, 1, EPI_BIAS, kStages>(L, ta, tb, tb, a, tiles);
+}
+
+
+// ---------------------------------------------------------------------------
+// MXFP4 weights with MXFP8 activations on the block-scaled tensor cores
+// ---------------------------------------------------------------------------
+// E4M3 rows [rows, K] bytes; boxes of 128 rows x 128 B, 128-byte swizzle.
+static cudaError_t make_tmap_e4m3(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kMx8BK), static_cast<cuuint32_t>(kBM)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Packed E2M1 weights [G, N, K/2] bytes viewed as super-rows of two weight rows:
+// {2K codes, N/2, G}; the 16U4_ALIGN16B type unpacks each 16 codes (8 B) into 16 B
+// of shared memory; boxes of 128 codes x box_rows super-rows, 128-byte swizzle.
+static cudaError_t make_tmap_e2m1_pairs(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t N, uint64_t G,
+                                        uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {2 * K, N / 2, G};
+  const cuuint64_t strides[2] = {K, K * (N / 2)};     // bytes: a super-row is 2 x K/2
+  const cuuint32_t box[3] = {128, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void*>(ptr), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int EPI, int TN, int NB, int STAGES>
+static cudaError_t launch_mx8(const Launch& L, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                              const Mx8Args& args, int64_t max_tiles) {
+  if (max_tiles <= 0) return cudaSuccess;
+  auto kern = grouped_gemm_mx8_kernel<EPI, TN, NB, STAGES>;
+  constexpr int smem = Mx8Layout<TN, NB>::smem_bytes(STAGES);
+  static_assert(smem <= 232448, "shared memory budget");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static std::mutex mu;
+  static uint64_t configured = 0;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (dev >= 64 || !((configured >> dev) & 1u)) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) configured |= uint64_t(1) << dev;
+    }
+  }
+  const int grid = static_cast<int>(std::min<int64_t>(max_tiles, L.num_sms));
+  pdl_launch(kern, dim3(grid), dim3(kMx8Threads), smem, L.stream, a, b0, b1, args);
+  count_launch();
+  return cudaGetLastError();
+}
+
+int mx8_sf_bytes_per_row(int K) { return mx8_sf_stride(K); }
+
+cudaError_t mx8_quant_rows(const Launch& L, int64_t T, int K, const void* x, uint8_t* xq, uint8_t* sf) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<int64_t>((T + 7) / 8, int64_t(L.num_sms) * 8));
+  pdl_launch(mx8_quant_rows_kernel, dim3(blocks), dim3(256), 0, L.stream, static_cast<const __nv_bfloat16*>(x),
+             static_cast<int>(T), K, mx8_sf_stride(K), xq, sf);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t mx8_weight_scales(const Launch& L, int D, int F, int E, const ExpertWeights& w, uint8_t* sf_gate,
+                              uint8_t* sf_up, uint8_t* sf_down) {
+  Mx8SfJob job{};
+  job.src[0] = w.s_gate; job.dst[0] = sf_gate; job.rows[0] = E * F; job.nblk[0] = D / 32; job.sfs[0] = mx8_sf_stride(D);
+  job.src[1] = w.s_up;   job.dst[1] = sf_up;   job.rows[1] = E * F; job.nblk[1] = D / 32; job.sfs[1] = mx8_sf_stride(D);
+  job.src[2] = w.s_down; job.dst[2] = sf_down; job.rows[2] = E * D; job.nblk[2] = F / 32; job.sfs[2] = mx8_sf_stride(F);
+  const int64_t most = std::max(int64_t(E) * F * job.sfs[0], int64_t(E) * D * job.sfs[2]);
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>((most + 255) / 256, int64_t(8) * L.num_sms)), 3);
+  pdl_launch(mx8_weight_sf_kernel, grid, dim3(256), 0, L.stream, job);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t expert_gateup_mx8(const Launch& L, int64_t R, int D, int F, int E, const uint8_t* xq,
+                              const uint8_t* sfx, const int32_t* expert_off, const ExpertWeights& w,
+                              const uint8_t* sf_gate, const uint8_t* sf_up, float limit, float alpha, uint8_t* hq,
+                              uint8_t* sfh) {
+  if (R == 0) return cudaSuccess;
+  CUtensorMap ta, tg, tu;
+  cudaError_t e;
+  if ((e = make_tmap_e4m3(&ta, xq, D, R)) != cudaSuccess) return e;
+  if ((e = make_tmap_e2m1_pairs(&tg, w.w_gate, D, F, E, kMx8TNGateUp / 2)) != cudaSuccess) return e;
+  if ((e = make_tmap_e2m1_pairs(&tu, w.w_up, D, F, E, kMx8TNGateUp / 2)) != cudaSuccess) return e;
+  Mx8Args a{};
+  a.group_off = expert_off;
+  a.num_groups = E;
+  a.m_total = static_cast<int>(R);
+  a.n_out = F;
+  a.k_dim = D;
+  a.sfa = sfx;
+  a.sfs_a = mx8_sf_stride(D);
+  a.sfw0 = sf_gate;
+  a.sfw1 = sf_up;
+  a.bias0 = w.b_gate;
+  a.bias1 = w.b_up;
+  a.limit = limit;
+  a.alpha = alpha;
+  a.gate_lo = 0.0f;
+  a.hq = hq;
+  a.sfh = sfh;
+  a.sfs_h = mx8_sf_stride(F);
+  a.wait_limit_ns = L.wait_limit_ns;
+  const int64_t tiles = max_row_blocks(R, E) * ((F + kMx8TNGateUp - 1) / kMx8TNGateUp);
+  return launch_mx8<EPI_SWIGLU, kMx8TNGateUp, 2, kMx8StagesGateUp>(L, ta, tg, tu, a, tiles);
+}
+
+cudaError_t expert_down_mx8(const Launch& L, int64_t R, int D, int F, int E, const uint8_t* hq, const uint8_t* sfh,
+                            const int32_t* expert_off, const ExpertWeights& w, const uint8_t* sf_down,
+                            const int32_t* slot_of_row, const float* topk_w, float* ys) {
+  if (R == 0) return cudaSuccess;
+  CUtensorMap ta, td;
+  cudaError_t e;
+  if ((e = make_tmap_e4m3(&ta, hq, F, R)) != cudaSuccess) return e;
+  if ((e = make_tmap_e2m1_pairs(&td, w.w_down, F, D, E, kMx8TNDown / 2)) != cudaSuccess) return e;
+  Mx8Args a{};
+  a.group_off = expert_off;
+  a.num_groups = E;
+  a.m_total = static_cast<int>(R);
+  a.n_out = D;
+  a.k_dim = F;
+  a.sfa = sfh;
+  a.sfs_a = mx8_sf_stride(F);
+  a.sfw0 = sf_down;
+  a.sfw1 = sf_down;
+  a.bias0 = w.b_down;
+  a.out = ys;
+  a.slot_of_row = slot_of_row;
+  a.topk_w = topk_w;
+  a.wait_limit_ns = L.wait_limit_ns;
+  const int64_t tiles = max_row_blocks(R, E) * ((D + kMx8TNDown - 1) / kMx8TNDown);
+  return launch_mx8<EPI_BIAS_WSCATTER, kMx8TNDown, 1, kMx8StagesDown>(L, ta, td, td, a, tiles);
+}
+
+// x_perm-style row gather of byte rows (row_bytes a multiple of 16): dst[r] = src[slot_of_row[r] / k].
+cudaError_t gather_rows(const Launch& L, const void* src, const int32_t* slot_of_row, int64_t R, int k, int64_t T,
+                        int row_bytes, void* dst) {
+  if (R == 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<int64_t>((R + 7) / 8, int64_t(L.num_sms) * 8));
+  pdl_launch(permute_gather_kernel, dim3(blocks), dim3(256), 0, L.stream, static_cast<const uint4*>(src), slot_of_row,
+             static_cast<int>(R), k, static_cast<int>(T), row_bytes / 16, static_cast<uint4*>(dst));
+  count_launch();
+  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -1,0 +1,594 @@
+// Expert GEMMs of the MXFP4 layer on the block-scaled tensor cores, with the
+// activations in MXFP8 (the layer's block-scaled numerics variant).
+//
+// The expert weights stay in the caller's MXFP4 form (E2M1 codes, one E8M0 scale
+// per 32 elements along K: "GPT-OSS 20B GGUF with MoE CPU Offloading", Model
+// Specifications; group size 32 for the 4-bit and MXFP8 formats: "Ollama
+// glm4_moe_lite.go", quantizationParams).  The activations -- x_perm for gate/up,
+// h for down -- are quantized to MXFP8 (E4M3 elements, one E8M0 scale per 32
+// elements along K; the scale 2^X is the smallest power of two with the block's
+// largest magnitude <= 448 * 2^X, so nothing saturates; elements round to nearest,
+// ties to even).  One tcgen05.mma.kind::mxf8f6f4.block_scale then multiplies
+// E4M3 by E2M1 with both operands' block scales applied by the tensor core, so
+// no weight is ever decoded in software.
+//
+// Operands in shared memory (128-byte swizzle, K-major, 128 K elements a stage):
+//   A  E4M3 rows by TMA (uint8 tensor map), 128 rows x 128 B.
+//   B  E2M1 rows by TMA with the 16U4_ALIGN16B data type: 16 packed codes (8 B)
+//      land in 16 B of shared memory, the layout the f8f6f4 MMA reads for 4-bit
+//      types.  That data type needs the row length to be a multiple of 128
+//      elements, which K = 2880 is not; so the tensor map views two consecutive
+//      weight rows as one "super-row" of 2K elements (2K = 5760 = 45 x 128 when
+//      K is a multiple of 64).  Even rows are read at element k, odd rows at K + k;
+//      a tile's rows n0..n0+TN-1 arrive as [TN/2 even rows][TN/2 odd rows], i.e.
+//      MMA column c holds weight row n0 + 2c (c < TN/2) or n0 + 2(c - TN/2) + 1.
+//      The last K block of an even row runs into the odd row's first codes; A is
+//      zero there (its tensor map ends at K), so those products vanish.
+//   SF the E8M0 scales, loaded by a warp of their own with 32-bit loads (four
+//      K blocks = one stage per load) from row-major copies padded to SFS bytes
+//      a row, stored into the 512-byte chunks tcgen05.cp copies to TMEM: byte
+//      16 (r % 32) + 4 (r / 32) + j holds row r's scale of the stage's block j,
+//      so TMEM lane r % 32 (replicated to all four lane quarters by .warpx4),
+//      column r / 32, byte j holds it -- the layout the block-scaled MMA reads
+//      with scale-factor id j.
+//
+// Roles (one CTA per SM, 224 threads): warp 0 TMA producer; warp 1 TMEM owner
+// and MMA issuer (tcgen05.cp of the stage's scales, then four MMAs of K = 32);
+// warps 2..5 epilogue; warp 6 scale loader.  Bounded waits throughout, as in
+// grouped_gemm.cuh.
+//
+// Epilogues:
+//   EPI_SWIGLU        NB = 2 (gate | up), TN = 96 features a tile (three 32-wide
+//                     blocks): the clipped SwiGLU, then h quantized to MXFP8 --
+//                     E4M3 codes into hq [R, F] and scales into sfh [R, SFS(F)].
+//   EPI_BIAS_WSCATTER NB = 1, TN = 240: ys[slot] = w[slot] * (C + b_d), fp32 rows
+//                     in slot order (the routing weight and un-permutation).
+#pragma once
+
+#include "grouped_gemm.cuh"
+
+namespace moe {
+
+constexpr int kMx8Threads = 224;
+constexpr int kMx8BK = 128;                 // K elements per stage (= 128 B of E4M3)
+constexpr int kMx8TNGateUp = 96;            // features per gate/up tile (F = 2880 = 30 x 96)
+constexpr int kMx8TNDown = 240;             // outputs per down tile (D = 2880 = 12 x 240)
+constexpr int kMx8StagesGateUp = 5;
+constexpr int kMx8StagesDown = 4;
+
+// bytes of scale per activation / weight row: four per 128-wide K block, rounded up to 16
+__host__ __device__ constexpr int mx8_sf_stride(int K) { return ((4 * ((K + 127) / 128)) + 15) / 16 * 16; }
+
+template <int TN, int NB>
+struct Mx8Layout {
+  static constexpr int N = TN * NB;                       // MMA N
+  static constexpr int A_BYTES = kBM * kMx8BK;            // 16 KB of E4M3
+  static constexpr int B_BYTES = N * kMx8BK;              // unpacked E2M1, 128 B a row
+  static constexpr int B_TX = N * kMx8BK / 2;             // bytes the TMA reads (packed)
+  static constexpr int SF_CHUNKS_B = (N + 127) / 128;
+  static constexpr int SF_BYTES = 512 * (1 + SF_CHUNKS_B);
+  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
+  static constexpr int EXTRA = 1024 + 4096;
+  static constexpr int smem_bytes(int stages) { return stages * STAGE_BYTES + EXTRA; }
+  // TMEM: accumulators at columns 0 and 256, then the scales of A (4 columns) and B
+  static constexpr int SFA_COL = 256 + (N + 3) / 4 * 4;
+  static constexpr int SFB_COL = SFA_COL + 4;
+  static_assert(N % 16 == 0 && N <= 256, "MMA N");
+  static_assert(SFB_COL + 4 * SF_CHUNKS_B <= kTmemCols, "scales fit beside the accumulators");
+  static_assert(TN % 2 == 0 && (TN / 2 * kMx8BK) % 1024 == 0, "even/odd halves start on swizzle atoms");
+};
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+// Instruction descriptor of kind::mxf8f6f4.block_scale: A E4M3 (0), B E2M1 (5),
+// E8M0 scales, K-major operands, fp32 accumulator; the scale-factor ids pick the
+// byte of each TMEM scale column the instruction uses.
+__host__ __device__ constexpr uint32_t make_idesc_mx8(int M, int N, uint32_t a_sf_id, uint32_t b_sf_id) {
+  return (b_sf_id << 4) | (0u << 7) | (5u << 10) | ((static_cast<uint32_t>(N) >> 3) << 17) | (1u << 23) |
+         ((static_cast<uint32_t>(M) >> 4) << 24) | (a_sf_id << 29);
+}
+
+__device__ __forceinline__ void tc_mma_mx8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// 32 rows x 16 B of shared memory to TMEM lanes 0..31 (and copies in lanes 32..127),
+// four consecutive 32-bit columns from `taddr`.
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of a 32 x 16 B scale chunk: no swizzle, 8-row core
+// matrices of 128 B one after another (both byte offsets 128).
+__device__ __forceinline__ uint64_t sf_chunk_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128 >> 4) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// The block scale exponent: the smallest X with amax <= 448 * 2^X (448 = 1.75 * 2^8),
+// read off amax's exponent and mantissa bits; -127 for zero and for amax < 2^-126.
+__device__ __forceinline__ int mx8_exponent(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int ef = static_cast<int>((b >> 23) & 0xFFu);
+  if (ef == 0) return -127;
+  const int X = (ef - 127) - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  return max(-127, min(127, X));
+}
+
+// 2^e for an integer e in [-127, 127], exactly.
+__device__ __forceinline__ float exp2_int(int e) {
+  return e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// Two floats to E4M3, round to nearest even (satfinite), `lo` in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Quantizes 32 values (one block) to MXFP8: 32 E4M3 bytes in q[8] (little-endian
+// words) and the E8M0 scale byte.
+__device__ __forceinline__ uint32_t mx8_quantize32(const float (&v)[32], uint32_t (&q)[8]) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+  const int X = mx8_exponent(amax);
+  const float inv = exp2_int(-X);
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const uint32_t p0 = e4m3x2(v[4 * w] * inv, v[4 * w + 1] * inv);
+    const uint32_t p1 = e4m3x2(v[4 * w + 2] * inv, v[4 * w + 3] * inv);
+    q[w] = p0 | (p1 << 16);
+  }
+  return static_cast<uint32_t>(X + 127);
+}
+
+// ---------------------------------------------------------------------------
+// activations to MXFP8: x [T, K] bf16 -> xq [T, K] E4M3, sf [T, SFS] E8M0
+// (scales of K/32 blocks, then 127 = 2^0 up to SFS so that padded K blocks scale
+// finite zeros).  One warp a row, a lane a 32-element block.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) mx8_quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int T, int K,
+                                                             int SFS, uint8_t* __restrict__ xq,
+                                                             uint8_t* __restrict__ sf) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int nb = K / 32;
+  for (int t = gw; t < T; t += nw) {
+    const __nv_bfloat16* row = x + static_cast<size_t>(t) * K;
+    for (int b = lane; b < nb; b += 32) {
+      float v[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float f[8];
+        load8<__nv_bfloat16>(row + 32 * b + 8 * c, f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[8 * c + j] = f[j];
+      }
+      uint32_t q[8];
+      const uint32_t s = mx8_quantize32(v, q);
+      uint4* dst = reinterpret_cast<uint4*>(xq + static_cast<size_t>(t) * K + 32 * b);
+      dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+      dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+      sf[static_cast<size_t>(t) * SFS + b] = static_cast<uint8_t>(s);
+    }
+    for (int b = nb + lane; b < SFS; b += 32) sf[static_cast<size_t>(t) * SFS + b] = 127;
+  }
+}
+
+// Weight scales [G, N, K/32] -> [G, N, SFS] (127 past K/32), for up to three matrices.
+struct Mx8SfJob {
+  const uint8_t* src[3];
+  uint8_t* dst[3];
+  int rows[3];     // G * N
+  int nblk[3];     // K / 32
+  int sfs[3];      // SFS(K)
+};
+__global__ void __launch_bounds__(256) mx8_weight_sf_kernel(Mx8SfJob job) {
+  pdl_enter();
+  const int m = blockIdx.y;
+  const int64_t total = static_cast<int64_t>(job.rows[m]) * job.sfs[m];
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / job.sfs[m];
+    const int c = static_cast<int>(i - r * job.sfs[m]);
+    job.dst[m][i] = c < job.nblk[m] ? job.src[m][r * job.nblk[m] + c] : static_cast<uint8_t>(127);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// arguments of the block-scaled GEMM
+// ---------------------------------------------------------------------------
+struct Mx8Args {
+  const int32_t* group_off;   // [G+1]
+  int num_groups;
+  int m_total;                // rows of A
+  int n_out;                  // weight rows per operand (F for gate/up, D for down)
+  int k_dim;                  // K
+  const uint8_t* sfa;         // [m_total, sfs_a] activation scales
+  int sfs_a;
+  const uint8_t* sfw0;        // [G, n_out, sfs_a] weight scales of B0 (and B1)
+  const uint8_t* sfw1;
+  const void* bias0;          // bf16 [G, n_out]
+  const void* bias1;
+  float limit, alpha, gate_lo;
+  uint8_t* hq;                // EPI_SWIGLU: [m_total, n_out] E4M3
+  uint8_t* sfh;               // EPI_SWIGLU: [m_total, sfs_h]
+  int sfs_h;
+  float* out;                 // EPI_BIAS_WSCATTER: [m_total, n_out] fp32, slot order
+  const int32_t* slot_of_row;
+  const float* topk_w;
+  unsigned long long wait_limit_ns;
+};
+
+// ---------------------------------------------------------------------------
+// epilogues (one thread = one accumulator row)
+// ---------------------------------------------------------------------------
+// gate/up: TMEM columns [gate even | gate odd | up even | up odd], TN / 2 each.
+template <int TN>
+__device__ __forceinline__ void mx8_epi_swiglu(uint32_t tbase, int row, bool rvalid, const TileInfo& ti,
+                                               const Mx8Args& a) {
+  constexpr int H = TN / 2;
+  const int F = a.n_out;
+  using T = __nv_bfloat16;
+  const T* bg = static_cast<const T*>(a.bias0) + static_cast<size_t>(ti.g) * F;
+  const T* bu = static_cast<const T*>(a.bias1) + static_cast<size_t>(ti.g) * F;
+#pragma unroll 1
+  for (int b = 0; b < TN / 32; ++b) {
+    const int f0 = ti.n0 + 32 * b;
+    float ge[16], go[16], ue[16], uo[16];
+    tmem_ld8(tbase + 16 * b, *reinterpret_cast<float(*)[8]>(ge));
+    tmem_ld8(tbase + 16 * b + 8, *reinterpret_cast<float(*)[8]>(ge + 8));
+    tmem_ld8(tbase + H + 16 * b, *reinterpret_cast<float(*)[8]>(go));
+    tmem_ld8(tbase + H + 16 * b + 8, *reinterpret_cast<float(*)[8]>(go + 8));
+    tmem_ld8(tbase + TN + 16 * b, *reinterpret_cast<float(*)[8]>(ue));
+    tmem_ld8(tbase + TN + 16 * b + 8, *reinterpret_cast<float(*)[8]>(ue + 8));
+    tmem_ld8(tbase + TN + H + 16 * b, *reinterpret_cast<float(*)[8]>(uo));
+    tmem_ld8(tbase + TN + H + 16 * b + 8, *reinterpret_cast<float(*)[8]>(uo + 8));
+    tmem_ld_wait();
+    if (!rvalid || f0 >= F) continue;
+    float h[32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float b0[8], b1[8];
+      load8<T>(bg + f0 + 8 * c, b0);
+      load8<T>(bu + f0 + 8 * c, b1);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = 8 * c + j;                       // feature f0 + i: even -> ge/ue, odd -> go/uo
+        const float g = (i & 1) ? go[i >> 1] : ge[i >> 1];
+        const float u = (i & 1) ? uo[i >> 1] : ue[i >> 1];
+        const float gc = fminf(fmaxf(g + b0[j], a.gate_lo), a.limit);
+        const float uc = fminf(fmaxf(u + b1[j], -a.limit), a.limit);
+        h[i] = __fdividef(gc * uc, 1.0f + __expf(-a.alpha * gc));
+      }
+    }
+    uint32_t q[8];
+    const uint32_t s = mx8_quantize32(h, q);
+    uint4* dst = reinterpret_cast<uint4*>(a.hq + static_cast<size_t>(row) * F + f0);
+    dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+    dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+    a.sfh[static_cast<size_t>(row) * a.sfs_h + f0 / 32] = static_cast<uint8_t>(s);
+  }
+  // scales of the padded K blocks of the down projection: 2^0 (finite, multiplying zeros)
+  if (rvalid && ti.n0 == 0)
+    for (int c = F / 32; c < a.sfs_h; ++c) a.sfh[static_cast<size_t>(row) * a.sfs_h + c] = 127;
+}
+
+// down: TMEM columns [even outputs | odd outputs], TN / 2 each; fp32 rows in slot order.
+template <int TN>
+__device__ __forceinline__ void mx8_epi_wscatter(uint32_t tbase, int row, bool rvalid, const TileInfo& ti,
+                                                 const Mx8Args& a) {
+  constexpr int H = TN / 2;
+  const int D = a.n_out;
+  using T = __nv_bfloat16;
+  float wv = 0.0f;
+  size_t orow = 0;
+  if (rvalid) {
+    const int s = a.slot_of_row[row];
+    if (s < 0 || s >= a.m_total) {
+      flag_error(DEVERR_BOUNDS);
+      rvalid = false;
+    } else {
+      orow = static_cast<size_t>(s);
+      wv = a.topk_w[s];
+    }
+  }
+  const T* bd = static_cast<const T*>(a.bias0) + static_cast<size_t>(ti.g) * D;
+#pragma unroll 1
+  for (int c = 0; c < H; c += 8) {
+    float ev[8], od[8];
+    tmem_ld8(tbase + c, ev);
+    tmem_ld8(tbase + H + c, od);
+    tmem_ld_wait();
+    const int d0 = ti.n0 + 2 * c;                     // outputs d0 .. d0 + 15
+    if (!rvalid || d0 >= D) continue;
+    float b[16];
+    load8<T>(bd + d0, *reinterpret_cast<float(*)[8]>(b));
+    load8<T>(bd + d0 + 8, *reinterpret_cast<float(*)[8]>(b + 8));
+    float o[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      o[2 * j] = wv * (ev[j] + b[2 * j]);
+      o[2 * j + 1] = wv * (od[j] + b[2 * j + 1]);
+    }
+    float* dst = a.out + orow * D + d0;
+    store8<float>(dst, *reinterpret_cast<float(*)[8]>(o));
+    store8<float>(dst + 8, *reinterpret_cast<float(*)[8]>(o + 8));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+template <int EPI, int TN, int NB, int STAGES>
+__global__ void __launch_bounds__(kMx8Threads, 1)
+    grouped_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                            const __grid_constant__ CUtensorMap tmB1, const Mx8Args args) {
+  pdl_enter();
+  using LY = Mx8Layout<TN, NB>;
+  constexpr int N = LY::N;
+  constexpr int H = TN / 2;
+  constexpr int KSTEPS = kMx8BK / 32;     // MMAs per stage (K = 32 each)
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * LY::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* never_flag = abort_flag + 1;
+  int* tile_off = never_flag + 2;              // [G+1]
+  int* goff = tile_off + (kMaxGroups + 2);     // [G+1]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = args.num_groups;
+  const int NT = (args.n_out + TN - 1) / TN;
+  const int KB = (args.k_dim + kMx8BK - 1) / kMx8BK;
+  const uint64_t lim = args.wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 2);    // the TMA producer's expect-tx arrival and the scale loader's
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&tfull[0], 1);
+    mbar_init(&tfull[1], 1);
+    mbar_init(&tempty[0], 128);
+    mbar_init(&tempty[1], 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *never_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) {
+    int bad = 0;
+    for (int g = lane; g <= G; g += 32) {
+      int v = args.group_off[g];
+      if (v < 0 || v > args.m_total) { bad = 1; v = min(max(v, 0), args.m_total); }
+      goff[g] = v;
+    }
+    __syncwarp();
+    int running = 0;
+    if (lane == 0) tile_off[0] = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int g = base + lane;
+      int cnt = 0;
+      if (g < G) {
+        const int rows = goff[g + 1] - goff[g];
+        if (rows < 0) bad = 1;
+        cnt = rows > 0 ? (rows + kBM - 1) / kBM : 0;
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      if (g < G) tile_off[g + 1] = running + incl;
+      running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) flag_error(DEVERR_BOUNDS);
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB0);
+      if (NB == 2) tma_prefetch_desc(&tmB1);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = tile_off[G] * NT;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint32_t tx_bytes = LY::A_BYTES + LY::B_TX;
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+        const TileInfo ti = decode_tile(i, tile_off, goff, G, NT, TN);
+        const int srow = ti.n0 / 2;                 // first super-row (two weight rows) of the tile
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], tx_bytes);
+          uint8_t* sa = smem + s * LY::STAGE_BYTES;
+          uint8_t* sb = sa + LY::A_BYTES;
+          const int k0 = kb * kMx8BK;
+          tma_load_2d(sa, &tmA, &full[s], k0, ti.m0);
+          tma_load_3d(sb, &tmB0, &full[s], k0, srow, ti.g);                              // even rows
+          tma_load_3d(sb + H * kMx8BK, &tmB0, &full[s], args.k_dim + k0, srow, ti.g);    // odd rows
+          if (NB == 2) {
+            tma_load_3d(sb + TN * kMx8BK, &tmB1, &full[s], k0, srow, ti.g);
+            tma_load_3d(sb + (TN + H) * kMx8BK, &tmB1, &full[s], args.k_dim + k0, srow, ti.g);
+          }
+          issued |= 1u << s;
+          issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag_error(DEVERR_TIMEOUT);
+      }
+      for (int q = 0; q < STAGES; ++q)
+        if ((issued >> q) & 1u)
+          if (!mbar_wait(&full[q], (issued_par >> q) & 1u, never_flag, kDrainLimitNs)) flag_error(DEVERR_TIMEOUT);
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ scale loader
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    const uint32_t one = 0x7F7F7F7Fu;   // four scales of 2^0
+    for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+      const TileInfo ti = decode_tile(i, tile_off, goff, G, NT, TN);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim))) { ok = false; break; }
+        uint32_t va[4], vb[2 * 4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {            // A rows lane + 32 j
+          const int r = ti.m0 + lane + 32 * j;
+          va[j] = r < args.m_total
+                      ? *reinterpret_cast<const uint32_t*>(args.sfa + static_cast<size_t>(r) * args.sfs_a + 4 * kb)
+                      : one;
+        }
+#pragma unroll
+        for (int j = 0; j < 4 * LY::SF_CHUNKS_B; ++j) {   // B positions lane + 32 j
+          const int c = lane + 32 * j;
+          uint32_t v = one;
+          if (c < N) {
+            const int op = c / TN, cc = c - op * TN;
+            const int n = ti.n0 + 2 * (cc % H) + cc / H;
+            if (n < args.n_out) {
+              const uint8_t* src = op == 0 ? args.sfw0 : args.sfw1;
+              v = *reinterpret_cast<const uint32_t*>(
+                  src + (static_cast<size_t>(ti.g) * args.n_out + n) * args.sfs_a + 4 * kb);
+            }
+          }
+          vb[j] = v;
+        }
+        uint8_t* sf = smem + s * LY::STAGE_BYTES + LY::A_BYTES + LY::B_BYTES;
+        *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(va[0], va[1], va[2], va[3]);
+#pragma unroll
+        for (int ch = 0; ch < LY::SF_CHUNKS_B; ++ch)
+          *reinterpret_cast<uint4*>(sf + 512 * (1 + ch) + 16 * lane) =
+              make_uint4(vb[4 * ch], vb[4 * ch + 1], vb[4 * ch + 2], vb[4 * ch + 3]);
+        fence_proxy_async_smem();   // the stores above are read by tcgen05.cp (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[s]);
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      flag_error(DEVERR_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(LY::SFA_COL);
+      const uint32_t sfb_t = tmem_base + static_cast<uint32_t>(LY::SFB_COL);
+      int s = 0, it = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; ok && i < total; i += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, lim)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag, lim)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * LY::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + LY::A_BYTES;
+          const uint32_t sf_addr = b_addr + LY::B_BYTES;
+          // the stage's scales into TMEM; tcgen05 operations of this thread run in order,
+          // so the previous stage's MMAs have read the old scales before these land
+          tc_cp_sf(sfa_t, sf_chunk_desc(sf_addr));
+#pragma unroll
+          for (int ch = 0; ch < LY::SF_CHUNKS_B; ++ch)
+            tc_cp_sf(sfb_t + 4 * ch, sf_chunk_desc(sf_addr + 512 * (1 + ch)));
+#pragma unroll
+          for (int kk = 0; kk < KSTEPS; ++kk) {
+            const uint32_t sel = static_cast<uint32_t>(kk) << 30;   // scale byte kk of each TMEM column
+            tc_mma_mx8(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32),
+                       make_idesc_mx8(kBM, N, kk, kk), sfa_t | sel, sfb_t | sel, (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag_error(DEVERR_TIMEOUT);
+      }
+      tc_commit(drain);
+      if (!mbar_wait(drain, 0, never_flag, kDrainLimitNs)) flag_error(DEVERR_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;
+    const int r_in_tile = quarter * 32 + lane;
+    int it = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < total; i += gridDim.x, ++it) {
+      const TileInfo ti = decode_tile(i, tile_off, goff, G, NT, TN);
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph, abort_flag, lim));
+      if (!got) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kAccStride);
+      const int row = ti.m0 + r_in_tile;
+      const bool rvalid = row < ti.m_end;
+      if constexpr (EPI == EPI_SWIGLU) mx8_epi_swiglu<TN>(tbase, row, rvalid, ti, args);
+      else mx8_epi_wscatter<TN>(tbase, row, rvalid, ti, args);
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      flag_error(DEVERR_TIMEOUT);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -64,6 +64,28 @@ cudaError_t combine_gather(const Launch& L, bool bf16, bool out_f32, int64_t T, 
 // y[t] = sum_j ys[t*k + j]   (ys fp32; y bf16 if out_bf16, else fp32)
 cudaError_t combine_slots(const Launch& L, bool out_bf16, int64_t T, int D, int k, const void* ys, void* y);
 
+// MXFP4 weights with MXFP8 activations on the block-scaled tensor cores.
+// Scale rows of K-long activation or weight rows: mx8_sf_bytes_per_row(K) bytes
+// (one E8M0 byte per 32 elements, then 127 = 2^0 for the padded K blocks).
+int mx8_sf_bytes_per_row(int K);
+// x [T, K] bf16 -> xq [T, K] E4M3 and sf [T, mx8_sf_bytes_per_row(K)].
+cudaError_t mx8_quant_rows(const Launch& L, int64_t T, int K, const void* x, uint8_t* xq, uint8_t* sf);
+// The caller's weight scales [E, N, K/32] as padded rows [E, N, mx8_sf_bytes_per_row(K)].
+cudaError_t mx8_weight_scales(const Launch& L, int D, int F, int E, const ExpertWeights& w, uint8_t* sf_gate,
+                              uint8_t* sf_up, uint8_t* sf_down);
+// gate/up + clipped SwiGLU: xq/sfx MXFP8 x_perm -> hq [R, F] E4M3 + sfh scale rows.
+cudaError_t expert_gateup_mx8(const Launch& L, int64_t R, int D, int F, int E, const uint8_t* xq,
+                              const uint8_t* sfx, const int32_t* expert_off, const ExpertWeights& w,
+                              const uint8_t* sf_gate, const uint8_t* sf_up, float limit, float alpha, uint8_t* hq,
+                              uint8_t* sfh);
+// down: ys[slot_of_row[r]] = topk_w[slot] * (hq[r] W_d^T + b_d), fp32.
+cudaError_t expert_down_mx8(const Launch& L, int64_t R, int D, int F, int E, const uint8_t* hq, const uint8_t* sfh,
+                            const int32_t* expert_off, const ExpertWeights& w, const uint8_t* sf_down,
+                            const int32_t* slot_of_row, const float* topk_w, float* ys);
+// dst[r] = src[slot_of_row[r] / k] for byte rows of row_bytes (a multiple of 16).
+cudaError_t gather_rows(const Launch& L, const void* src, const int32_t* slot_of_row, int64_t R, int k, int64_t T,
+                        int row_bytes, void* dst);
+
 // The same two projections with MXFP4 expert weights, dequantised inside the GEMM mainloop.
 // The kernels read the E8M0 scales from a copy relaid as [E][ceil(K/64)][N][2]
 // (mx_scale_bytes each), written by mx_scale_relayout on the same stream.

@@ -43,19 +43,24 @@ moe_status_t check_cfg(const moe_config_t* c) {
   if (c == nullptr) return MOE_ERR_INVALID_ARG;
   const int D = c->hidden_size, F = c->intermediate_size, E = c->num_local_experts, k = c->num_experts_per_tok;
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
-  if (c->wfmt != MOE_W_DENSE && c->wfmt != MOE_W_MXFP4) return MOE_ERR_INVALID_ARG;
+  if (c->wfmt != MOE_W_DENSE && c->wfmt != MOE_W_MXFP4 && c->wfmt != MOE_W_MXFP4_A8) return MOE_ERR_INVALID_ARG;
   if (E < 1 || E > 256 || k < 1 || k > 8 || k > E) return MOE_ERR_INVALID_ARG;
   if (D <= 0 || F <= 0 || D > (1 << 20) || F > (1 << 20)) return MOE_ERR_INVALID_ARG;
-  const int mult = c->wfmt == MOE_W_MXFP4 ? 32 : 16;
+  const int mult = c->wfmt == MOE_W_DENSE ? 16 : 32;
   if (D % mult != 0 || F % mult != 0) return MOE_ERR_INVALID_ARG;
   if (!std::isfinite(c->swiglu_limit) || !(c->swiglu_limit > 0.0f) || !std::isfinite(c->swiglu_alpha))
     return MOE_ERR_INVALID_ARG;
   if (c->y_f32 != 0 && c->y_f32 != 1) return MOE_ERR_INVALID_ARG;
   if (c->h_split != 0 && c->h_split != 1) return MOE_ERR_INVALID_ARG;
-  if (c->wfmt == MOE_W_MXFP4 && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-  if (c->wfmt == MOE_W_MXFP4 && c->h_split != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->wfmt != MOE_W_DENSE && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (c->wfmt != MOE_W_DENSE && c->h_split != 0) return MOE_ERR_UNSUPPORTED;
+  // the block-scaled path reads two weight rows as one 2K-code row, a multiple of 128 codes
+  if (c->wfmt == MOE_W_MXFP4_A8 && (D % 64 != 0 || F % 64 != 0)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
+
+bool mxfp4_weights(const moe_config_t* c) { return c->wfmt == MOE_W_MXFP4 || c->wfmt == MOE_W_MXFP4_A8; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // h kept as two bf16 halves (bf16 layers; fp32 layers keep h in fp32 and ignore the flag)
 int h_halves(const moe_config_t* c) { return (c->dtype == MOE_BF16 && c->h_split != 0) ? 2 : 1; }
@@ -120,6 +125,51 @@ Layout layout(const moe_config_t* c, int64_t T) {
   return L;
 }
 
+// Workspace of moe_layer_forward with MOE_W_MXFP4_A8: the maps, then x and x_perm in
+// MXFP8 (E4M3 rows and scale rows), h in MXFP8, the weighted fp32 rows, and the
+// weights' scale rows padded for 32-bit loads.
+struct LayoutA8 {
+  size_t ids, w, off, ros, sor, pscr, xq, sfx, xpq, sfa, hq, sfh, ys, sfw_g, sfw_u, sfw_d, rpart, total;
+};
+
+LayoutA8 layout_a8(const moe_config_t* c, int64_t T) {
+  const size_t R = size_t(T) * c->num_experts_per_tok;
+  const size_t D = c->hidden_size, F = c->intermediate_size, E = c->num_local_experts;
+  const size_t sd = moe::mx8_sf_bytes_per_row(c->hidden_size), sf = moe::mx8_sf_bytes_per_row(c->intermediate_size);
+  LayoutA8 L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.ids = take(R * 4);
+  L.w = take(R * 4);
+  L.off = take((E + 1) * 4);
+  L.ros = take(R * 4);
+  L.sor = take(R * 4);
+  L.pscr = take(moe::permute_scratch_words(T, c->num_local_experts) * 4);
+  L.xq = take(size_t(T) * D);
+  L.sfx = take(size_t(T) * sd);
+  L.xpq = take(R * D);
+  L.sfa = take(R * sd);
+  // the router's K-split partial logits are dead before gate/up writes hq: they share it
+  const size_t rpart_bytes = moe::router_partial_bytes(T, c->num_local_experts);
+  L.hq = take(R * F > rpart_bytes ? R * F : rpart_bytes);
+  L.rpart = L.hq;
+  L.sfh = take(R * sf);
+  L.ys = take(R * D * 4);
+  L.sfw_g = take(E * F * sd);
+  L.sfw_u = take(E * F * sd);
+  L.sfw_d = take(E * D * sf);
+  L.total = o;
+  return L;
+}
+
+size_t layer_ws_bytes(const moe_config_t* c, int64_t T) {
+  return c->wfmt == MOE_W_MXFP4_A8 ? layout_a8(c, T).total : layout(c, T).total;
+}
+
 bool get_launch(void* stream, Launch* L) {
   static std::mutex mu;
   static int sms[64] = {0};
@@ -147,7 +197,10 @@ bool weights_ok(const moe_config_t* c, const moe_expert_weights_t* w) {
   if (w == nullptr) return false;
   if (!ptr_ok(w->w_gate) || !ptr_ok(w->w_up) || !ptr_ok(w->w_down)) return false;
   if (!ptr_ok(w->b_gate) || !ptr_ok(w->b_up) || !ptr_ok(w->b_down)) return false;
-  if (c->wfmt == MOE_W_MXFP4 && (!ptr_ok(w->s_gate) || !ptr_ok(w->s_up) || !ptr_ok(w->s_down))) return false;
+  if (mxfp4_weights(c) && (!ptr_ok(w->s_gate) || !ptr_ok(w->s_up) || !ptr_ok(w->s_down))) return false;
+  // the 4-bit tensor maps of the block-scaled path need 32-byte aligned rows
+  if (c->wfmt == MOE_W_MXFP4_A8 && (!aligned32(w->w_gate) || !aligned32(w->w_up) || !aligned32(w->w_down)))
+    return false;
   return true;
 }
 
@@ -317,6 +370,56 @@ GlmLayout glm_layout(const moe_config_t* c, const moe_glm_params_t* p, int64_t T
   return L;
 }
 
+// moe_layer_forward with MXFP4 weights and MXFP8 activations (arguments already checked)
+moe_status_t layer_forward_a8(const moe_config_t* cfg, const Launch& L, int64_t T, const void* x,
+                              const void* w_router, const void* b_router, const moe_expert_weights_t* weights, void* y,
+                              int32_t* topk_ids_out, float* topk_w_out, void* ws) {
+  const LayoutA8 LY = layout_a8(cfg, T);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t*>(base + LY.ids);
+  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(base + LY.w);
+  int32_t* eoff = reinterpret_cast<int32_t*>(base + LY.off);
+  int32_t* ros = reinterpret_cast<int32_t*>(base + LY.ros);
+  int32_t* sor = reinterpret_cast<int32_t*>(base + LY.sor);
+  int32_t* pscr = reinterpret_cast<int32_t*>(base + LY.pscr);
+  const int D = cfg->hidden_size, F = cfg->intermediate_size, E = cfg->num_local_experts,
+            k = cfg->num_experts_per_tok;
+  const int64_t R = T * k;
+  const moe::ExpertWeights wt = to_internal(weights);
+
+  stage_mark(ST_ROUTER, true, L.stream);
+  if (moe::router_topk(L, true, T, D, E, k, x, w_router, b_router, ids, w,
+                       reinterpret_cast<float*>(base + LY.rpart)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  stage_mark(ST_ROUTER, false, L.stream);
+  stage_mark(ST_DISPATCH, true, L.stream);
+  if (moe::permute(L, true, T, D, E, k, ids, nullptr, eoff, ros, sor, nullptr, pscr) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (moe::mx8_quant_rows(L, T, D, x, base + LY.xq, base + LY.sfx) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::gather_rows(L, base + LY.xq, sor, R, k, T, D, base + LY.xpq) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::gather_rows(L, base + LY.sfx, sor, R, k, T, moe::mx8_sf_bytes_per_row(D), base + LY.sfa) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  stage_mark(ST_DISPATCH, false, L.stream);
+  stage_mark(ST_GATEUP, true, L.stream);
+  if (moe::mx8_weight_scales(L, D, F, E, wt, base + LY.sfw_g, base + LY.sfw_u, base + LY.sfw_d) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (moe::expert_gateup_mx8(L, R, D, F, E, base + LY.xpq, base + LY.sfa, eoff, wt, base + LY.sfw_g,
+                             base + LY.sfw_u, cfg->swiglu_limit, cfg->swiglu_alpha, base + LY.hq,
+                             base + LY.sfh) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  stage_mark(ST_GATEUP, false, L.stream);
+  stage_mark(ST_DOWN, true, L.stream);
+  float* ys = reinterpret_cast<float*>(base + LY.ys);
+  if (moe::expert_down_mx8(L, R, D, F, E, base + LY.hq, base + LY.sfh, eoff, wt, base + LY.sfw_d, sor, w, ys) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  stage_mark(ST_DOWN, false, L.stream);
+  stage_mark(ST_COMBINE, true, L.stream);
+  const moe_status_t s = cuda_status(moe::combine_slots(L, out_bf16(cfg), T, D, k, ys, y));
+  stage_mark(ST_COMBINE, false, L.stream);
+  return s;
+}
+
 }  // namespace
 
 extern "C" {
@@ -350,7 +453,7 @@ size_t moe_expert_ffn_workspace_size(const moe_config_t* cfg, int64_t T) {
 
 size_t moe_workspace_size(const moe_config_t* cfg, int64_t T) {
   if (check_cfg(cfg) != MOE_OK || !check_T(T, cfg->num_experts_per_tok)) return size_t(-1);
-  return layout(cfg, T).total;
+  return layer_ws_bytes(cfg, T);
 }
 
 moe_status_t moe_router_topk(const moe_config_t* cfg, int64_t T, const void* x, const void* w_router,
@@ -420,6 +523,7 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, int64_t T, const void* x_pe
   if (!ptr_ok(x_perm) || !ptr_ok(expert_off) || !ptr_ok(h) || !ptr_ok(y_perm) || !weights_ok(cfg, weights))
     return MOE_ERR_INVALID_ARG;
   if ((s = check_variant(cfg)) != MOE_OK) return s;
+  if (cfg->wfmt == MOE_W_MXFP4_A8) return MOE_ERR_UNSUPPORTED;   // its activations never leave MXFP8
   const size_t need = ffn_ws_bytes(cfg, T);
   if (need > 0 && (ws == nullptr || !aligned16(ws) || ws_bytes < need)) return MOE_ERR_WORKSPACE;
   Launch L;
@@ -452,10 +556,12 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x
   if ((topk_ids_out != nullptr && !aligned16(topk_ids_out)) || (topk_w_out != nullptr && !aligned16(topk_w_out)))
     return MOE_ERR_INVALID_ARG;
   if ((s = check_variant(cfg)) != MOE_OK) return s;
-  const Layout LY = layout(cfg, T);
-  if (ws == nullptr || !aligned16(ws) || ws_bytes < LY.total) return MOE_ERR_WORKSPACE;
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < layer_ws_bytes(cfg, T)) return MOE_ERR_WORKSPACE;
   Launch L;
   if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
+  if (cfg->wfmt == MOE_W_MXFP4_A8)
+    return layer_forward_a8(cfg, L, T, x, w_router, b_router, weights, y, topk_ids_out, topk_w_out, ws);
+  const Layout LY = layout(cfg, T);
 
   uint8_t* base = static_cast<uint8_t*>(ws);
   int32_t* ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t*>(base + LY.ids);
@@ -485,6 +591,17 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x
   s = cuda_status(moe::combine_slots(L, out_bf16(cfg), T, D, k, ys, y));
   stage_mark(ST_COMBINE, false, L.stream);
   return s;
+}
+
+int32_t moe_mxfp8_scale_stride(int32_t K) { return K > 0 ? moe::mx8_sf_bytes_per_row(K) : -1; }
+
+moe_status_t moe_quantize_mxfp8(int64_t rows, int32_t K, const void* x, uint8_t* xq, uint8_t* sf, void* stream) {
+  if (rows < 0 || K <= 0 || K % 32 != 0 || K > (1 << 20) || rows > (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!ptr_ok(x) || !ptr_ok(xq) || !ptr_ok(sf)) return MOE_ERR_INVALID_ARG;
+  Launch L;
+  if (!get_launch(stream, &L)) return MOE_ERR_CUDA;
+  return cuda_status(moe::mx8_quant_rows(L, rows, K, x, xq, sf));
 }
 
 moe_status_t moe_last_device_error(void) {
