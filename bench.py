@@ -52,6 +52,9 @@ def parse_args():
     p.add_argument("--no-mxfp4", action="store_true", help="skip the MXFP4-weight layer")
     p.add_argument("--no-skewed", action="store_true", help="skip the GPT-OSS-120B-shaped skewed layer")
     p.add_argument("--no-glm", action="store_true", help="skip the GLM4-MoE-Lite variant layer")
+    p.add_argument("--wfmt", choices=("mxfp4", "mxfp4_a8"), default=None,
+                   help="MXFP4 workloads: decode the weights in the GEMM mainloop (mxfp4, the default) or "
+                        "multiply them on the block-scaled tensor cores with MXFP8 activations (mxfp4_a8)")
     p.add_argument("--h-split", action="store_true",
                    help="keep the SwiGLU output as two bf16 halves between the expert GEMMs (h_split)")
     return p.parse_args()
@@ -67,10 +70,10 @@ def measured_peaks():
     return dict(bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, hbm_gbs=6650.0, source="fallback")
 
 
-def config_of(spec, n_gpus, h_split=False):
+def config_of(spec, n_gpus, h_split=False, wfmt=None):
     return {"workload": spec.name, "h_split": h_split, "T_per_gpu": spec.T, "hidden_size": spec.D, "intermediate_size": spec.F,
             "num_local_experts": spec.E, "num_experts_per_tok": spec.k, "swiglu_limit": spec.limit,
-            "expert_weights": spec.wfmt, "global_tokens": spec.T * n_gpus,
+            "expert_weights": wfmt or spec.wfmt, "global_tokens": spec.T * n_gpus,
             "parallelism": f"dp{n_gpus} (independent replicas)",
             "l2": "inputs larger than L2: every step streams all expert weights "
                   f"({expert_weight_bytes(spec) / 1e9:.2f} GB) through HBM"}
@@ -228,7 +231,9 @@ def run_ours(args, rank, world, local_rank):
     if rank > 0:   # each replica routes its own tokens
         layer["x"] = W.make_layer(spec, seed=rank, with_experts=False)["x"]
     d = api.upload_layer(layer, dev)
-    cfg = api.config_from_spec(spec, h_split=args.h_split)
+    if args.wfmt is not None and spec.wfmt != "mxfp4":
+        raise SystemExit("--wfmt applies to MXFP4 workloads")
+    cfg = api.config_from_spec(spec, h_split=args.h_split, wfmt=args.wfmt)
     moe = api.MoELayer(cfg, d["w_router"], d["b_router"], api.expert_weights_from(d))
     x, T = d["x"], spec.T
     y = torch.empty_like(x)
@@ -346,7 +351,7 @@ def run_ours(args, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if spec.dtype == "bf16" else "f32",
             "data": "synthetic (seeded random-init weights and activations of the GPT-OSS-20B MoE layer shape)",
-            "config": config_of(spec, world, args.h_split),
+            "config": config_of(spec, world, args.h_split, args.wfmt),
             "tflops": flops / (ms_step / 1e3) / 1e12,
             "roofline": {"bound": "tensor", "kernel": "gateup_swiglu_gemm", "achieved": achieved,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
@@ -594,9 +599,28 @@ def mxfp4_sweep(api, dev, stream, steps):
     if api.last_device_error() != 0:
         raise RuntimeError("device error word set during the MXFP4 steps")
     gu_tf = 4.0 * spec.R * spec.D * spec.F / (stage["gateup_swiglu_gemm"] * 1e-6) / 1e12
-    return {"workload": spec.name, "T": spec.T, "us_per_step": us, "tokens/s": spec.T / (us * 1e-6),
-            "stage_us": stage, "gateup_tflops": gu_tf, "gateup_frac": gu_tf / peaks["bf16_tflops"],
-            "weight_bytes": 3 * spec.E * spec.D * spec.F // 2 + 3 * spec.E * spec.D * spec.F // 32}
+    out = {"workload": spec.name, "T": spec.T, "us_per_step": us, "tokens/s": spec.T / (us * 1e-6),
+           "stage_us": stage, "gateup_tflops": gu_tf, "gateup_frac": gu_tf / peaks["bf16_tflops"],
+           "weight_bytes": 3 * spec.E * spec.D * spec.F // 2 + 3 * spec.E * spec.D * spec.F // 32}
+    # the same weights on the block-scaled tensor cores with MXFP8 activations (MOE_W_MXFP4_A8);
+    # its peak is the f8f6f4 rate, twice the bf16 one (nominal 4.5 against 2.25 PFLOP/s dense)
+    moe8 = api.MoELayer(api.config_from_spec(spec, wfmt="mxfp4_a8"), d["w_router"], d["b_router"], moe.experts)
+    for _ in range(3):
+        moe8(x, y=y)
+    torch.cuda.synchronize()
+    us8 = 1e3 * timed_steps(lambda: moe8(x, y=y), stream, steps)
+    stage8 = {k: 1e3 * v for k, v in stage_times(lambda: moe8(x, y=y), stream, steps).items()}
+    if api.last_device_error() != 0:
+        raise RuntimeError("device error word set during the MXFP4 x MXFP8 steps")
+    fl = 2.0 * spec.R * spec.D * spec.F
+    gu8 = 2 * fl / (stage8["gateup_swiglu_gemm"] * 1e-6) / 1e12
+    dn8 = fl / (stage8["down_combine_gemm"] * 1e-6) / 1e12
+    peak8 = 2.0 * peaks["bf16_tflops"]
+    out["a8"] = {"wfmt": "mxfp4_a8", "us_per_step": us8, "tokens/s": spec.T / (us8 * 1e-6), "stage_us": stage8,
+                 "gateup_tflops": gu8, "down_tflops": dn8, "peak_tflops": peak8,
+                 "peak_source": peaks["source"] + " bf16 burst x 2 (nominal f8f6f4 : bf16 rate)",
+                 "gateup_frac": gu8 / peak8, "down_frac": dn8 / peak8}
+    return out
 
 
 def reduce_max(v: float, device) -> float:

@@ -88,8 +88,8 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
  * elements rounded to nearest, ties to even.  A numerics variant of the layer
  * (the pages name MXFP8 and its group size 32, "Ollama glm4_moe_lite.go",
  * quantizationParams); its results differ from MOE_W_MXFP4 by that
- * quantization.  Needs D and F multiples of 64 and weight pointers 32-byte
- * aligned; moe_layer_forward only (moe_expert_ffn returns MOE_ERR_UNSUPPORTED). */
+ * quantization.  Same weight layout and sizes as MOE_W_MXFP4;
+ * moe_layer_forward only (moe_expert_ffn returns MOE_ERR_UNSUPPORTED). */
 typedef enum { MOE_W_DENSE = 0, MOE_W_MXFP4 = 1, MOE_W_MXFP4_A8 = 2 } moe_wfmt_t;
 
 /* Field names follow the GPT-OSS Config (hidden_size, num_local_experts,

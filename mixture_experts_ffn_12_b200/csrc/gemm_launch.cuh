@@ -583,20 +583,19 @@ static cudaError_t make_tmap_e4m3(CUtensorMap* m, const void* ptr, uint64_t K, u
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// Packed E2M1 weights [G, N, K/2] bytes viewed as super-rows of two weight rows:
-// {2K codes, N/2, G}; the 16U4_ALIGN16B type unpacks each 16 codes (8 B) into 16 B
-// of shared memory; boxes of 128 codes x box_rows super-rows, 128-byte swizzle.
-static cudaError_t make_tmap_e2m1_pairs(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t N, uint64_t G,
-                                        uint32_t box_rows) {
+// Packed E2M1 weights [G, N, K/2] bytes as they are; boxes of 64 B (128 codes) x box_rows,
+// no swizzle (the converter warps widen them into the swizzled tile).
+static cudaError_t make_tmap_e2m1(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t N, uint64_t G,
+                                  uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return cudaErrorNotSupported;
-  const cuuint64_t dims[3] = {2 * K, N / 2, G};
-  const cuuint64_t strides[2] = {K, K * (N / 2)};     // bytes: a super-row is 2 x K/2
-  const cuuint32_t box[3] = {128, box_rows, 1};
+  const cuuint64_t dims[3] = {K / 2, N, G};
+  const cuuint64_t strides[2] = {K / 2, (K / 2) * N};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kMx8BK / 2), box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void*>(ptr), dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -657,8 +656,8 @@ cudaError_t expert_gateup_mx8(const Launch& L, int64_t R, int D, int F, int E, c
   CUtensorMap ta, tg, tu;
   cudaError_t e;
   if ((e = make_tmap_e4m3(&ta, xq, D, R)) != cudaSuccess) return e;
-  if ((e = make_tmap_e2m1_pairs(&tg, w.w_gate, D, F, E, kMx8TNGateUp / 2)) != cudaSuccess) return e;
-  if ((e = make_tmap_e2m1_pairs(&tu, w.w_up, D, F, E, kMx8TNGateUp / 2)) != cudaSuccess) return e;
+  if ((e = make_tmap_e2m1(&tg, w.w_gate, D, F, E, kMx8TNGateUp)) != cudaSuccess) return e;
+  if ((e = make_tmap_e2m1(&tu, w.w_up, D, F, E, kMx8TNGateUp)) != cudaSuccess) return e;
   Mx8Args a{};
   a.group_off = expert_off;
   a.num_groups = E;
@@ -689,7 +688,7 @@ cudaError_t expert_down_mx8(const Launch& L, int64_t R, int D, int F, int E, con
   CUtensorMap ta, td;
   cudaError_t e;
   if ((e = make_tmap_e4m3(&ta, hq, F, R)) != cudaSuccess) return e;
-  if ((e = make_tmap_e2m1_pairs(&td, w.w_down, F, D, E, kMx8TNDown / 2)) != cudaSuccess) return e;
+  if ((e = make_tmap_e2m1(&td, w.w_down, F, D, E, kMx8TNDown)) != cudaSuccess) return e;
   Mx8Args a{};
   a.group_off = expert_off;
   a.num_groups = E;

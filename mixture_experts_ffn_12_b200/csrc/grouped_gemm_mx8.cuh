@@ -14,16 +14,13 @@
 //
 // Operands in shared memory (128-byte swizzle, K-major, 128 K elements a stage):
 //   A  E4M3 rows by TMA (uint8 tensor map), 128 rows x 128 B.
-//   B  E2M1 rows by TMA with the 16U4_ALIGN16B data type: 16 packed codes (8 B)
-//      land in 16 B of shared memory, the layout the f8f6f4 MMA reads for 4-bit
-//      types.  That data type needs the row length to be a multiple of 128
-//      elements, which K = 2880 is not; so the tensor map views two consecutive
-//      weight rows as one "super-row" of 2K elements (2K = 5760 = 45 x 128 when
-//      K is a multiple of 64).  Even rows are read at element k, odd rows at K + k;
-//      a tile's rows n0..n0+TN-1 arrive as [TN/2 even rows][TN/2 odd rows], i.e.
-//      MMA column c holds weight row n0 + 2c (c < TN/2) or n0 + 2(c - TN/2) + 1.
-//      The last K block of an even row runs into the odd row's first codes; A is
-//      zero there (its tensor map ends at K), so those products vanish.
+//   B  the f8f6f4 MMA reads 4-bit operands with each 16 codes (8 B) in 16 B of
+//      shared memory, the upper 8 B unused.  The packed rows (64 B per 128 codes)
+//      arrive by a plain byte TMA in a staging area; four converter warps widen
+//      every 8 B to 16 B (zeros above) into the 128-byte-swizzled tile the MMA
+//      reads -- byte moves only, any K that is a multiple of 32.  (TMA's own
+//      unpacking type needs row lengths and start coordinates in 128-code units,
+//      which K = 2880 is not.)
 //   SF the E8M0 scales, loaded by a warp of their own with 32-bit loads (four
 //      K blocks = one stage per load) from row-major copies padded to SFS bytes
 //      a row, stored into the 512-byte chunks tcgen05.cp copies to TMEM: byte
@@ -32,10 +29,10 @@
 //      column r / 32, byte j holds it -- the layout the block-scaled MMA reads
 //      with scale-factor id j.
 //
-// Roles (one CTA per SM, 224 threads): warp 0 TMA producer; warp 1 TMEM owner
+// Roles (one CTA per SM, 352 threads): warp 0 TMA producer; warp 1 TMEM owner
 // and MMA issuer (tcgen05.cp of the stage's scales, then four MMAs of K = 32);
-// warps 2..5 epilogue; warp 6 scale loader.  Bounded waits throughout, as in
-// grouped_gemm.cuh.
+// warps 2..5 epilogue; warp 6 scale loader; warps 7..10 converters.  Bounded
+// waits throughout, as in grouped_gemm.cuh.
 //
 // Epilogues:
 //   EPI_SWIGLU        NB = 2 (gate | up), TN = 96 features a tile (three 32-wide
@@ -49,12 +46,13 @@
 
 namespace moe {
 
-constexpr int kMx8Threads = 224;
+constexpr int kMx8Threads = 352;
+constexpr int kMx8ConvWarps = 4;
 constexpr int kMx8BK = 128;                 // K elements per stage (= 128 B of E4M3)
 constexpr int kMx8TNGateUp = 96;            // features per gate/up tile (F = 2880 = 30 x 96)
 constexpr int kMx8TNDown = 240;             // outputs per down tile (D = 2880 = 12 x 240)
-constexpr int kMx8StagesGateUp = 5;
-constexpr int kMx8StagesDown = 4;
+constexpr int kMx8StagesGateUp = 4;
+constexpr int kMx8StagesDown = 3;
 
 // bytes of scale per activation / weight row: four per 128-wide K block, rounded up to 16
 __host__ __device__ constexpr int mx8_sf_stride(int K) { return ((4 * ((K + 127) / 128)) + 15) / 16 * 16; }
@@ -63,11 +61,11 @@ template <int TN, int NB>
 struct Mx8Layout {
   static constexpr int N = TN * NB;                       // MMA N
   static constexpr int A_BYTES = kBM * kMx8BK;            // 16 KB of E4M3
-  static constexpr int B_BYTES = N * kMx8BK;              // unpacked E2M1, 128 B a row
-  static constexpr int B_TX = N * kMx8BK / 2;             // bytes the TMA reads (packed)
+  static constexpr int B_BYTES = N * kMx8BK;              // widened E2M1, 128 B a row
+  static constexpr int P_BYTES = N * kMx8BK / 2;          // packed E2M1 as the TMA delivers it
   static constexpr int SF_CHUNKS_B = (N + 127) / 128;
   static constexpr int SF_BYTES = 512 * (1 + SF_CHUNKS_B);
-  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
+  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + P_BYTES + SF_BYTES + 1023) / 1024 * 1024;
   static constexpr int EXTRA = 1024 + 4096;
   static constexpr int smem_bytes(int stages) { return stages * STAGE_BYTES + EXTRA; }
   // TMEM: accumulators at columns 0 and 256, then the scales of A (4 columns) and B
@@ -75,7 +73,8 @@ struct Mx8Layout {
   static constexpr int SFB_COL = SFA_COL + 4;
   static_assert(N % 16 == 0 && N <= 256, "MMA N");
   static_assert(SFB_COL + 4 * SF_CHUNKS_B <= kTmemCols, "scales fit beside the accumulators");
-  static_assert(TN % 2 == 0 && (TN / 2 * kMx8BK) % 1024 == 0, "even/odd halves start on swizzle atoms");
+  static_assert((TN * kMx8BK) % 1024 == 0, "the up operand starts on a swizzle atom");
+  static_assert((N * 8) % (32 * kMx8ConvWarps) == 0, "16-byte chunks split evenly over the converters");
 };
 
 // ---------------------------------------------------------------------------
@@ -238,11 +237,10 @@ struct Mx8Args {
 // ---------------------------------------------------------------------------
 // epilogues (one thread = one accumulator row)
 // ---------------------------------------------------------------------------
-// gate/up: TMEM columns [gate even | gate odd | up even | up odd], TN / 2 each.
+// gate/up: TMEM columns [gate 0..TN-1 | up TN..2TN-1].
 template <int TN>
 __device__ __forceinline__ void mx8_epi_swiglu(uint32_t tbase, int row, bool rvalid, const TileInfo& ti,
                                                const Mx8Args& a) {
-  constexpr int H = TN / 2;
   const int F = a.n_out;
   using T = __nv_bfloat16;
   const T* bg = static_cast<const T*>(a.bias0) + static_cast<size_t>(ti.g) * F;
@@ -250,15 +248,12 @@ __device__ __forceinline__ void mx8_epi_swiglu(uint32_t tbase, int row, bool rva
 #pragma unroll 1
   for (int b = 0; b < TN / 32; ++b) {
     const int f0 = ti.n0 + 32 * b;
-    float ge[16], go[16], ue[16], uo[16];
-    tmem_ld8(tbase + 16 * b, *reinterpret_cast<float(*)[8]>(ge));
-    tmem_ld8(tbase + 16 * b + 8, *reinterpret_cast<float(*)[8]>(ge + 8));
-    tmem_ld8(tbase + H + 16 * b, *reinterpret_cast<float(*)[8]>(go));
-    tmem_ld8(tbase + H + 16 * b + 8, *reinterpret_cast<float(*)[8]>(go + 8));
-    tmem_ld8(tbase + TN + 16 * b, *reinterpret_cast<float(*)[8]>(ue));
-    tmem_ld8(tbase + TN + 16 * b + 8, *reinterpret_cast<float(*)[8]>(ue + 8));
-    tmem_ld8(tbase + TN + H + 16 * b, *reinterpret_cast<float(*)[8]>(uo));
-    tmem_ld8(tbase + TN + H + 16 * b + 8, *reinterpret_cast<float(*)[8]>(uo + 8));
+    float g[32], u[32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      tmem_ld8(tbase + 32 * b + 8 * c, *reinterpret_cast<float(*)[8]>(g + 8 * c));
+      tmem_ld8(tbase + TN + 32 * b + 8 * c, *reinterpret_cast<float(*)[8]>(u + 8 * c));
+    }
     tmem_ld_wait();
     if (!rvalid || f0 >= F) continue;
     float h[32];
@@ -269,12 +264,9 @@ __device__ __forceinline__ void mx8_epi_swiglu(uint32_t tbase, int row, bool rva
       load8<T>(bu + f0 + 8 * c, b1);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int i = 8 * c + j;                       // feature f0 + i: even -> ge/ue, odd -> go/uo
-        const float g = (i & 1) ? go[i >> 1] : ge[i >> 1];
-        const float u = (i & 1) ? uo[i >> 1] : ue[i >> 1];
-        const float gc = fminf(fmaxf(g + b0[j], a.gate_lo), a.limit);
-        const float uc = fminf(fmaxf(u + b1[j], -a.limit), a.limit);
-        h[i] = __fdividef(gc * uc, 1.0f + __expf(-a.alpha * gc));
+        const float gc = fminf(fmaxf(g[8 * c + j] + b0[j], a.gate_lo), a.limit);
+        const float uc = fminf(fmaxf(u[8 * c + j] + b1[j], -a.limit), a.limit);
+        h[8 * c + j] = __fdividef(gc * uc, 1.0f + __expf(-a.alpha * gc));
       }
     }
     uint32_t q[8];
@@ -289,11 +281,10 @@ __device__ __forceinline__ void mx8_epi_swiglu(uint32_t tbase, int row, bool rva
     for (int c = F / 32; c < a.sfs_h; ++c) a.sfh[static_cast<size_t>(row) * a.sfs_h + c] = 127;
 }
 
-// down: TMEM columns [even outputs | odd outputs], TN / 2 each; fp32 rows in slot order.
+// down: TMEM columns 0..TN-1 = outputs n0..n0+TN-1; fp32 rows in slot order.
 template <int TN>
 __device__ __forceinline__ void mx8_epi_wscatter(uint32_t tbase, int row, bool rvalid, const TileInfo& ti,
                                                  const Mx8Args& a) {
-  constexpr int H = TN / 2;
   const int D = a.n_out;
   using T = __nv_bfloat16;
   float wv = 0.0f;
@@ -310,31 +301,25 @@ __device__ __forceinline__ void mx8_epi_wscatter(uint32_t tbase, int row, bool r
   }
   const T* bd = static_cast<const T*>(a.bias0) + static_cast<size_t>(ti.g) * D;
 #pragma unroll 1
-  for (int c = 0; c < H; c += 8) {
-    float ev[8], od[8];
-    tmem_ld8(tbase + c, ev);
-    tmem_ld8(tbase + H + c, od);
+  for (int c = 0; c < TN; c += 8) {
+    float v[8];
+    tmem_ld8(tbase + c, v);
     tmem_ld_wait();
-    const int d0 = ti.n0 + 2 * c;                     // outputs d0 .. d0 + 15
+    const int d0 = ti.n0 + c;
     if (!rvalid || d0 >= D) continue;
-    float b[16];
-    load8<T>(bd + d0, *reinterpret_cast<float(*)[8]>(b));
-    load8<T>(bd + d0 + 8, *reinterpret_cast<float(*)[8]>(b + 8));
-    float o[16];
+    float b[8];
+    load8<T>(bd + d0, b);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      o[2 * j] = wv * (ev[j] + b[2 * j]);
-      o[2 * j + 1] = wv * (od[j] + b[2 * j + 1]);
-    }
-    float* dst = a.out + orow * D + d0;
-    store8<float>(dst, *reinterpret_cast<float(*)[8]>(o));
-    store8<float>(dst + 8, *reinterpret_cast<float(*)[8]>(o + 8));
+    for (int j = 0; j < 8; ++j) v[j] = wv * (v[j] + b[j]);
+    store8<float>(a.out + orow * D + d0, v);
   }
 }
 
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
+// tmA: E4M3 activations [m_total, K]; tmB0 / tmB1: packed E2M1 weights [G, n_out, K/2] bytes,
+// boxes of 64 B (128 codes) x TN rows.
 template <int EPI, int TN, int NB, int STAGES>
 __global__ void __launch_bounds__(kMx8Threads, 1)
     grouped_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
@@ -342,13 +327,13 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
   pdl_enter();
   using LY = Mx8Layout<TN, NB>;
   constexpr int N = LY::N;
-  constexpr int H = TN / 2;
   constexpr int KSTEPS = kMx8BK / 32;     // MMAs per stage (K = 32 each)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * LY::STAGE_BYTES);
-  uint64_t* empty = full + STAGES;
+  uint64_t* conv = full + STAGES;              // widened B tile and scales in place
+  uint64_t* empty = conv + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
@@ -357,6 +342,11 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
   int* never_flag = abort_flag + 1;
   int* tile_off = never_flag + 2;              // [G+1]
   int* goff = tile_off + (kMaxGroups + 2);     // [G+1]
+  // a stage: [A | B widened | B packed | scales]
+  auto stage_a = [&](int s) { return smem + s * LY::STAGE_BYTES; };
+  auto stage_b = [&](int s) { return smem + s * LY::STAGE_BYTES + LY::A_BYTES; };
+  auto stage_p = [&](int s) { return smem + s * LY::STAGE_BYTES + LY::A_BYTES + LY::B_BYTES; };
+  auto stage_sf = [&](int s) { return smem + s * LY::STAGE_BYTES + LY::A_BYTES + LY::B_BYTES + LY::P_BYTES; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -367,7 +357,8 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 2);    // the TMA producer's expect-tx arrival and the scale loader's
+      mbar_init(&full[s], 1);
+      mbar_init(&conv[s], kMx8ConvWarps + 1);   // the converter warps and the scale loader
       mbar_init(&empty[s], 1);
     }
     mbar_init(&tfull[0], 1);
@@ -426,26 +417,18 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint32_t tx_bytes = LY::A_BYTES + LY::B_TX;
+      const uint32_t tx_bytes = LY::A_BYTES + LY::P_BYTES;
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_par = 0;
       bool ok = true;
       for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
         const TileInfo ti = decode_tile(i, tile_off, goff, G, NT, TN);
-        const int srow = ti.n0 / 2;                 // first super-row (two weight rows) of the tile
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], tx_bytes);
-          uint8_t* sa = smem + s * LY::STAGE_BYTES;
-          uint8_t* sb = sa + LY::A_BYTES;
-          const int k0 = kb * kMx8BK;
-          tma_load_2d(sa, &tmA, &full[s], k0, ti.m0);
-          tma_load_3d(sb, &tmB0, &full[s], k0, srow, ti.g);                              // even rows
-          tma_load_3d(sb + H * kMx8BK, &tmB0, &full[s], args.k_dim + k0, srow, ti.g);    // odd rows
-          if (NB == 2) {
-            tma_load_3d(sb + TN * kMx8BK, &tmB1, &full[s], k0, srow, ti.g);
-            tma_load_3d(sb + (TN + H) * kMx8BK, &tmB1, &full[s], args.k_dim + k0, srow, ti.g);
-          }
+          tma_load_2d(stage_a(s), &tmA, &full[s], kb * kMx8BK, ti.m0);
+          tma_load_3d(stage_p(s), &tmB0, &full[s], kb * (kMx8BK / 2), ti.n0, ti.g);
+          if (NB == 2) tma_load_3d(stage_p(s) + TN * (kMx8BK / 2), &tmB1, &full[s], kb * (kMx8BK / 2), ti.n0, ti.g);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -460,6 +443,42 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
           if (!mbar_wait(&full[q], (issued_par >> q) & 1u, never_flag, kDrainLimitNs)) flag_error(DEVERR_TIMEOUT);
     }
     __syncwarp();
+  } else if (warp >= 7) {
+    // ------------------------------------------------------------ converters: packed -> widened B
+    // 16-byte chunk q of the tile (row q / 8, chunk q % 8) takes the 8 packed bytes of its 16 codes
+    // and zeros; chunk c of row r sits at r * 128 + ((c ^ (r % 8)) * 16) under the 128-byte swizzle
+    const int ct = threadIdx.x - 7 * 32;
+    constexpr int PER = N * 8 / (32 * kMx8ConvWarps);
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim))) { ok = false; break; }
+        const uint8_t* src = stage_p(s);
+        uint8_t* dst = stage_b(s);
+        uint2 v[PER];
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+          const int q = ct + j * 32 * kMx8ConvWarps;
+          v[j] = *reinterpret_cast<const uint2*>(src + 8 * q);
+        }
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+          const int q = ct + j * 32 * kMx8ConvWarps;
+          const int r = q >> 3, c = q & 7;
+          *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(v[j].x, v[j].y, 0u, 0u);
+        }
+        fence_proxy_async_smem();   // the widened tile is read by the tensor core (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&conv[s]);
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      flag_error(DEVERR_TIMEOUT);
+    }
   } else if (warp == 6) {
     // ------------------------------------------------------------ scale loader
     int s = 0;
@@ -470,7 +489,7 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
       const TileInfo ti = decode_tile(i, tile_off, goff, G, NT, TN);
       for (int kb = 0; kb < KB; ++kb) {
         if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim))) { ok = false; break; }
-        uint32_t va[4], vb[2 * 4];
+        uint32_t va[4], vb[4 * LY::SF_CHUNKS_B];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {            // A rows lane + 32 j
           const int r = ti.m0 + lane + 32 * j;
@@ -483,8 +502,8 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
           const int c = lane + 32 * j;
           uint32_t v = one;
           if (c < N) {
-            const int op = c / TN, cc = c - op * TN;
-            const int n = ti.n0 + 2 * (cc % H) + cc / H;
+            const int op = c / TN;
+            const int n = ti.n0 + (c - op * TN);
             if (n < args.n_out) {
               const uint8_t* src = op == 0 ? args.sfw0 : args.sfw1;
               v = *reinterpret_cast<const uint32_t*>(
@@ -493,7 +512,7 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
           }
           vb[j] = v;
         }
-        uint8_t* sf = smem + s * LY::STAGE_BYTES + LY::A_BYTES + LY::B_BYTES;
+        uint8_t* sf = stage_sf(s);
         *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(va[0], va[1], va[2], va[3]);
 #pragma unroll
         for (int ch = 0; ch < LY::SF_CHUNKS_B; ++ch)
@@ -501,7 +520,7 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
               make_uint4(vb[4 * ch], vb[4 * ch + 1], vb[4 * ch + 2], vb[4 * ch + 3]);
         fence_proxy_async_smem();   // the stores above are read by tcgen05.cp (async proxy)
         __syncwarp();
-        if (lane == 0) mbar_arrive(&full[s]);
+        if (lane == 0) mbar_arrive(&conv[s]);
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
     }
@@ -524,11 +543,12 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&full[s], ph, abort_flag, lim)) { ok = false; break; }
+          // the converters waited for the TMA (A, packed B) before arriving here
+          if (!mbar_wait(&conv[s], ph, abort_flag, lim)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * LY::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + LY::A_BYTES;
-          const uint32_t sf_addr = b_addr + LY::B_BYTES;
+          const uint32_t a_addr = smem_u32(stage_a(s));
+          const uint32_t b_addr = smem_u32(stage_b(s));
+          const uint32_t sf_addr = smem_u32(stage_sf(s));
           // the stage's scales into TMEM; tcgen05 operations of this thread run in order,
           // so the previous stage's MMAs have read the old scales before these land
           tc_cp_sf(sfa_t, sf_chunk_desc(sf_addr));

@@ -54,13 +54,10 @@ moe_status_t check_cfg(const moe_config_t* c) {
   if (c->h_split != 0 && c->h_split != 1) return MOE_ERR_INVALID_ARG;
   if (c->wfmt != MOE_W_DENSE && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (c->wfmt != MOE_W_DENSE && c->h_split != 0) return MOE_ERR_UNSUPPORTED;
-  // the block-scaled path reads two weight rows as one 2K-code row, a multiple of 128 codes
-  if (c->wfmt == MOE_W_MXFP4_A8 && (D % 64 != 0 || F % 64 != 0)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
 bool mxfp4_weights(const moe_config_t* c) { return c->wfmt == MOE_W_MXFP4 || c->wfmt == MOE_W_MXFP4_A8; }
-bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // h kept as two bf16 halves (bf16 layers; fp32 layers keep h in fp32 and ignore the flag)
 int h_halves(const moe_config_t* c) { return (c->dtype == MOE_BF16 && c->h_split != 0) ? 2 : 1; }
@@ -198,9 +195,6 @@ bool weights_ok(const moe_config_t* c, const moe_expert_weights_t* w) {
   if (!ptr_ok(w->w_gate) || !ptr_ok(w->w_up) || !ptr_ok(w->w_down)) return false;
   if (!ptr_ok(w->b_gate) || !ptr_ok(w->b_up) || !ptr_ok(w->b_down)) return false;
   if (mxfp4_weights(c) && (!ptr_ok(w->s_gate) || !ptr_ok(w->s_up) || !ptr_ok(w->s_down))) return false;
-  // the 4-bit tensor maps of the block-scaled path need 32-byte aligned rows
-  if (c->wfmt == MOE_W_MXFP4_A8 && (!aligned32(w->w_gate) || !aligned32(w->w_up) || !aligned32(w->w_down)))
-    return false;
   return true;
 }
 

@@ -166,19 +166,20 @@ def test_h_split_workspace_and_variant_check(lib):
 
 
 def test_block_scaled_variant_checks(lib):
-    """MXFP4 weights with MXFP8 activations: bf16 layers, D and F multiples of 64, no h_split,
+    """MXFP4 weights with MXFP8 activations: bf16 layers, D and F multiples of 32, no h_split,
     moe_layer_forward only; the quantizer's argument checks; all before any launch."""
     a8 = _lib.MOE_W_MXFP4_A8
     assert lib.moe_config_check(ctypes.byref(cfg(wfmt=a8))) == _lib.MOE_OK
-    assert lib.moe_config_check(ctypes.byref(cfg(wfmt=a8, hidden_size=2880 - 32))) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.moe_config_check(ctypes.byref(cfg(wfmt=a8, hidden_size=2880 - 32))) == _lib.MOE_OK
+    assert lib.moe_config_check(ctypes.byref(cfg(wfmt=a8, hidden_size=2880 - 16))) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_config_check(ctypes.byref(cfg(wfmt=a8, dtype=_lib.MOE_F32))) == _lib.MOE_ERR_UNSUPPORTED
     assert lib.moe_config_check(ctypes.byref(cfg(wfmt=a8, h_split=1))) == _lib.MOE_ERR_UNSUPPORTED
     p = ctypes.c_void_p(0x10000)
     w = _lib.MoeExpertWeights(*([0x10000] * 9))
     assert lib.moe_expert_ffn(ctypes.byref(cfg(wfmt=a8)), 8, p, p, ctypes.byref(w), p, p, None, 0, None) == \
         _lib.MOE_ERR_UNSUPPORTED
-    w16 = _lib.MoeExpertWeights(*([0x10010] + [0x10000] * 8))      # 16- but not 32-byte aligned codes
-    assert lib.moe_layer_forward(ctypes.byref(cfg(wfmt=a8)), 8, p, p, p, ctypes.byref(w16), p, None, None, p,
+    w8 = _lib.MoeExpertWeights(*([0x10008] + [0x10000] * 8))       # codes not 16-byte aligned
+    assert lib.moe_layer_forward(ctypes.byref(cfg(wfmt=a8)), 8, p, p, p, ctypes.byref(w8), p, None, None, p,
                                  1 << 40, None) == _lib.MOE_ERR_INVALID_ARG
     c, big = cfg(wfmt=a8), 1 << 40
     assert lib.moe_workspace_size(ctypes.byref(c), 8192) != _lib.SIZE_INVALID

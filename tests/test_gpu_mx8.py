@@ -34,7 +34,8 @@ def _bf16_rows(rng, rows, K):
     a = rng.normal(0, 1, (rows, K)) * np.exp(rng.normal(0, 3, (rows, 1)))
     a[0, :32] = 0.0                                   # an all-zero block
     a[1, :32] = 448.0 * 2.0 ** -5                     # largest magnitude exactly 448 * 2^X
-    a[1, 32:64] = 1.75 * 2.0 ** np.arange(-16, 16)    # one block spanning many binades
+    if K >= 64:
+        a[1, 32:64] = 1.75 * 2.0 ** np.arange(-16, 16)    # one block spanning many binades
     a[2, :32] = 1e-30                                 # bf16 values far below the E4M3 range of 2^0
     return W.f32_to_bf16_bits(a.astype(np.float32))
 
@@ -109,23 +110,3 @@ def test_layer_a8_full_size_sampled(api):
     toks = np.unique(np.concatenate([[0, spec.T - 1], rng.choice(spec.T, 46, replace=False),
                                      sor[off[0]:off[1]][:16] // spec.k]))
     _check(api, spec, layer, toks)
-
-
-def test_layer_a8_rejects_unaligned_weights(api):
-    """The 4-bit tensor maps need 32-byte aligned weight rows: a 16-byte aligned pointer is refused
-    before anything is launched."""
-    from mixture_experts_ffn_12_b200 import _lib
-    spec = MX8_SMALL
-    d = api.upload_layer(layer_for(spec))
-    ew = api.expert_weights_from(d)
-    buf = torch.empty(ew.w_gate.numel() + 32, dtype=torch.uint8, device="cuda")
-    off = (16 - buf.data_ptr() % 32) % 32                 # start at 16 mod 32
-    shifted = buf[off:off + ew.w_gate.numel()].view(ew.w_gate.shape)
-    shifted.copy_(ew.w_gate)
-    ew.w_gate = shifted
-    lib = _lib.load()
-    before = lib.moe_launch_count()
-    with pytest.raises(api.MoeError) as e:
-        api.layer_forward(api.config_from_spec(spec, wfmt="mxfp4_a8"), d["x"], d["w_router"], d["b_router"], ew)
-    assert e.value.code == _lib.MOE_ERR_INVALID_ARG
-    assert lib.moe_launch_count() == before
