@@ -29,10 +29,15 @@
 //      column r / 32, byte j holds it -- the layout the block-scaled MMA reads
 //      with scale-factor id j.
 //
-// Roles (one CTA per SM, 352 threads): warp 0 TMA producer; warp 1 TMEM owner
+// Roles (one CTA per SM, 448 threads): warp 0 TMA producer; warp 1 TMEM owner
 // and MMA issuer (tcgen05.cp of the stage's scales, then four MMAs of K = 32);
-// warps 2..5 epilogue; warp 6 scale loader; warps 7..10 converters.  Bounded
-// waits throughout, as in grouped_gemm.cuh.
+// warps 2..5 epilogue; warps 7..10 converters; warps 6, 11, 12, 13 scale loaders
+// (a stage's scales are one round trip of 32-bit loads, longer than its MMAs: four
+// loaders keep four round trips in flight).  Loader j owns the ring slots s with
+// s % 4 == j and feeds every use of them in order, so each of its parity waits is
+// for the release of a use it fed itself (a loader that took uses of a slot in turn
+// with other loaders could wait two phases ahead, where a parity wait passes at
+// once).  Bounded waits throughout, as in grouped_gemm.cuh.
 //
 // Epilogues:
 //   EPI_SWIGLU        NB = 2 (gate | up), TN = 96 features a tile (three 32-wide
@@ -46,8 +51,9 @@
 
 namespace moe {
 
-constexpr int kMx8Threads = 352;
+constexpr int kMx8Threads = 448;
 constexpr int kMx8ConvWarps = 4;
+constexpr int kMx8SfWarps = 4;
 constexpr int kMx8BK = 128;                 // K elements per stage (= 128 B of E4M3)
 constexpr int kMx8TNGateUp = 96;            // features per gate/up tile (F = 2880 = 30 x 96)
 constexpr int kMx8TNDown = 240;             // outputs per down tile (D = 2880 = 12 x 240)
@@ -443,7 +449,7 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
           if (!mbar_wait(&full[q], (issued_par >> q) & 1u, never_flag, kDrainLimitNs)) flag_error(DEVERR_TIMEOUT);
     }
     __syncwarp();
-  } else if (warp >= 7) {
+  } else if (warp >= 7 && warp <= 10) {
     // ------------------------------------------------------------ converters: packed -> widened B
     // 16-byte chunk q of the tile (row q / 8, chunk q % 8) takes the 8 packed bytes of its 16 codes
     // and zeros; chunk c of row r sits at r * 128 + ((c ^ (r % 8)) * 16) under the 128-byte swizzle
@@ -479,15 +485,18 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
       *abort_flag = 1;
       flag_error(DEVERR_TIMEOUT);
     }
-  } else if (warp == 6) {
-    // ------------------------------------------------------------ scale loader
-    int s = 0;
-    uint32_t ph = 0;
+  } else if (warp == 6 || warp > 10) {
+    // ------------------------------------------------------------ scale loaders (slot s: loader s % 4)
+    const int me = warp == 6 ? 0 : warp - 10;
+    int n = 0;                                    // stages of this CTA so far
     bool ok = true;
     const uint32_t one = 0x7F7F7F7Fu;   // four scales of 2^0
     for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
       const TileInfo ti = decode_tile(i, tile_off, goff, G, NT, TN);
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = 0; kb < KB; ++kb, ++n) {
+        const int s = n % STAGES;
+        if (s % kMx8SfWarps != me) continue;
+        const uint32_t ph = static_cast<uint32_t>(n / STAGES) & 1u;
         if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim))) { ok = false; break; }
         uint32_t va[4], vb[4 * LY::SF_CHUNKS_B];
 #pragma unroll
@@ -521,7 +530,6 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
         fence_proxy_async_smem();   // the stores above are read by tcgen05.cp (async proxy)
         __syncwarp();
         if (lane == 0) mbar_arrive(&conv[s]);
-        if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
     }
     if (!ok && lane == 0) {
