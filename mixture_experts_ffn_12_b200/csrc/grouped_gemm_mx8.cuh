@@ -487,50 +487,72 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
     }
   } else if (warp == 6 || warp > 10) {
     // ------------------------------------------------------------ scale loaders (slot s: loader s % 4)
+    // Step n of this CTA is K block n % KB of its (n / KB)-th tile.  A loader issues the
+    // global loads of its next step before it waits for the current step's slot, so the
+    // load round trip overlaps the wait.
     const int me = warp == 6 ? 0 : warp - 10;
-    int n = 0;                                    // stages of this CTA so far
-    bool ok = true;
     const uint32_t one = 0x7F7F7F7Fu;   // four scales of 2^0
-    for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
-      const TileInfo ti = decode_tile(i, tile_off, goff, G, NT, TN);
-      for (int kb = 0; kb < KB; ++kb, ++n) {
-        const int s = n % STAGES;
-        if (s % kMx8SfWarps != me) continue;
-        const uint32_t ph = static_cast<uint32_t>(n / STAGES) & 1u;
-        if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim))) { ok = false; break; }
-        uint32_t va[4], vb[4 * LY::SF_CHUNKS_B];
+    const int my_tiles = static_cast<int>(blockIdx.x) < total
+                             ? (total - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                                   static_cast<int>(gridDim.x)
+                             : 0;
+    const int steps = my_tiles * KB;
+    auto owned_from = [&](int n) {      // first step >= n whose slot this loader owns
+      while (n < steps && (n % STAGES) % kMx8SfWarps != me) ++n;
+      return n;
+    };
+    constexpr int NB4 = 4 * LY::SF_CHUNKS_B;
+    auto load = [&](int n, uint32_t (&va)[4], uint32_t (&vb)[NB4]) {
+      const TileInfo ti = decode_tile(static_cast<int>(blockIdx.x) + (n / KB) * static_cast<int>(gridDim.x),
+                                      tile_off, goff, G, NT, TN);
+      const int kb = n % KB;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {            // A rows lane + 32 j
-          const int r = ti.m0 + lane + 32 * j;
-          va[j] = r < args.m_total
-                      ? *reinterpret_cast<const uint32_t*>(args.sfa + static_cast<size_t>(r) * args.sfs_a + 4 * kb)
-                      : one;
-        }
-#pragma unroll
-        for (int j = 0; j < 4 * LY::SF_CHUNKS_B; ++j) {   // B positions lane + 32 j
-          const int c = lane + 32 * j;
-          uint32_t v = one;
-          if (c < N) {
-            const int op = c / TN;
-            const int n = ti.n0 + (c - op * TN);
-            if (n < args.n_out) {
-              const uint8_t* src = op == 0 ? args.sfw0 : args.sfw1;
-              v = *reinterpret_cast<const uint32_t*>(
-                  src + (static_cast<size_t>(ti.g) * args.n_out + n) * args.sfs_a + 4 * kb);
-            }
-          }
-          vb[j] = v;
-        }
-        uint8_t* sf = stage_sf(s);
-        *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(va[0], va[1], va[2], va[3]);
-#pragma unroll
-        for (int ch = 0; ch < LY::SF_CHUNKS_B; ++ch)
-          *reinterpret_cast<uint4*>(sf + 512 * (1 + ch) + 16 * lane) =
-              make_uint4(vb[4 * ch], vb[4 * ch + 1], vb[4 * ch + 2], vb[4 * ch + 3]);
-        fence_proxy_async_smem();   // the stores above are read by tcgen05.cp (async proxy)
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&conv[s]);
+      for (int j = 0; j < 4; ++j) {            // A rows lane + 32 j
+        const int r = ti.m0 + lane + 32 * j;
+        va[j] = r < args.m_total
+                    ? *reinterpret_cast<const uint32_t*>(args.sfa + static_cast<size_t>(r) * args.sfs_a + 4 * kb)
+                    : one;
       }
+#pragma unroll
+      for (int j = 0; j < NB4; ++j) {          // B positions lane + 32 j
+        const int c = lane + 32 * j;
+        uint32_t v = one;
+        if (c < N) {
+          const int op = c / TN;
+          const int nrow = ti.n0 + (c - op * TN);
+          if (nrow < args.n_out) {
+            const uint8_t* src = op == 0 ? args.sfw0 : args.sfw1;
+            v = *reinterpret_cast<const uint32_t*>(
+                src + (static_cast<size_t>(ti.g) * args.n_out + nrow) * args.sfs_a + 4 * kb);
+          }
+        }
+        vb[j] = v;
+      }
+    };
+    bool ok = true;
+    uint32_t va[4], vb[NB4], na[4], nb[NB4];
+    int n = owned_from(0);
+    if (n < steps) load(n, va, vb);
+    while (ok && n < steps) {
+      const int next = owned_from(n + 1);
+      if (next < steps) load(next, na, nb);
+      const int s = n % STAGES;
+      const uint32_t ph = static_cast<uint32_t>(n / STAGES) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim))) { ok = false; break; }
+      uint8_t* sf = stage_sf(s);
+      *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(va[0], va[1], va[2], va[3]);
+#pragma unroll
+      for (int ch = 0; ch < LY::SF_CHUNKS_B; ++ch)
+        *reinterpret_cast<uint4*>(sf + 512 * (1 + ch) + 16 * lane) =
+            make_uint4(vb[4 * ch], vb[4 * ch + 1], vb[4 * ch + 2], vb[4 * ch + 3]);
+      fence_proxy_async_smem();   // the stores above are read by tcgen05.cp (async proxy)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&conv[s]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) va[j] = na[j];
+#pragma unroll
+      for (int j = 0; j < NB4; ++j) vb[j] = nb[j];
+      n = next;
     }
     if (!ok && lane == 0) {
       *abort_flag = 1;
