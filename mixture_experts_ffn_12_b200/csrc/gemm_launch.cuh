@@ -641,7 +641,7 @@ cudaError_t mx8_weight_scales(const Launch& L, int D, int F, int E, const Expert
   job.src[0] = w.s_gate; job.dst[0] = sf_gate; job.rows[0] = E * F; job.nblk[0] = D / 32; job.sfs[0] = mx8_sf_stride(D);
   job.src[1] = w.s_up;   job.dst[1] = sf_up;   job.rows[1] = E * F; job.nblk[1] = D / 32; job.sfs[1] = mx8_sf_stride(D);
   job.src[2] = w.s_down; job.dst[2] = sf_down; job.rows[2] = E * D; job.nblk[2] = F / 32; job.sfs[2] = mx8_sf_stride(F);
-  const int64_t most = std::max(int64_t(E) * F * job.sfs[0], int64_t(E) * D * job.sfs[2]);
+  const int64_t most = std::max(int64_t(E) * F * job.sfs[0], int64_t(E) * D * job.sfs[2]) / 16;   // chunks
   const dim3 grid(static_cast<unsigned>(std::min<int64_t>((most + 255) / 256, int64_t(8) * L.num_sms)), 3);
   pdl_launch(mx8_weight_sf_kernel, grid, dim3(256), 0, L.stream, job);
   count_launch();

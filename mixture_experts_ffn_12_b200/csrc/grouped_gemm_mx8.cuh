@@ -203,15 +203,33 @@ struct Mx8SfJob {
   int nblk[3];     // K / 32
   int sfs[3];      // SFS(K)
 };
+// One thread per 16-byte chunk of an output row (the rows are tens of bytes; 32-bit indices).
 __global__ void __launch_bounds__(256) mx8_weight_sf_kernel(Mx8SfJob job) {
   pdl_enter();
   const int m = blockIdx.y;
-  const int64_t total = static_cast<int64_t>(job.rows[m]) * job.sfs[m];
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / job.sfs[m];
-    const int c = static_cast<int>(i - r * job.sfs[m]);
-    job.dst[m][i] = c < job.nblk[m] ? job.src[m][r * job.nblk[m] + c] : static_cast<uint8_t>(127);
+  const int rows = m == 0 ? job.rows[0] : m == 1 ? job.rows[1] : job.rows[2];
+  const int nblk = m == 0 ? job.nblk[0] : m == 1 ? job.nblk[1] : job.nblk[2];
+  const int sfs = m == 0 ? job.sfs[0] : m == 1 ? job.sfs[1] : job.sfs[2];
+  const uint8_t* src = m == 0 ? job.src[0] : m == 1 ? job.src[1] : job.src[2];
+  uint8_t* dst = m == 0 ? job.dst[0] : m == 1 ? job.dst[1] : job.dst[2];
+  const int cpr = sfs / 16;
+  const int total = rows * cpr;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const int r = i / cpr;
+    const int c = i - r * cpr;
+    const uint8_t* s = src + static_cast<size_t>(r) * nblk;
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int j = 16 * c + 4 * q + b;
+        v |= (j < nblk ? static_cast<uint32_t>(s[j]) : 127u) << (8 * b);
+      }
+      w[q] = v;
+    }
+    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * sfs + 16 * c) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 

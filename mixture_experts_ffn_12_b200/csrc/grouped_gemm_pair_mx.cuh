@@ -106,18 +106,19 @@ struct MxScaleJob {
 __global__ void __launch_bounds__(256) mx_scale_relayout_kernel(MxScaleJob job) {
   pdl_enter();
   const int m = blockIdx.y;
-  const int N = job.rows[m], K = job.kdim[m];
+  const int N = m == 0 ? job.rows[0] : m == 1 ? job.rows[1] : job.rows[2];
+  const int K = m == 0 ? job.kdim[0] : m == 1 ? job.kdim[1] : job.kdim[2];
+  const uint8_t* src = m == 0 ? job.src[0] : m == 1 ? job.src[1] : job.src[2];
+  uint16_t* dst = reinterpret_cast<uint16_t*>(m == 0 ? job.dst[0] : m == 1 ? job.dst[1] : job.dst[2]);
   const int KS = K / 32, KB = (K + 63) / 64;
-  const int64_t total = static_cast<int64_t>(job.groups) * KB * N;
-  const uint8_t* src = job.src[m];
-  uint16_t* dst = reinterpret_cast<uint16_t*>(job.dst[m]);
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int n = static_cast<int>(i % N);
-    const int64_t gk = i / N;
-    const int kb = static_cast<int>(gk % KB);
-    const int64_t g = gk / KB;
-    const uint8_t* row = src + (g * N + n) * KS;
+  // 32-bit index arithmetic: the config check keeps groups * KB * N (and twice it) below 2^31
+  const int total = job.groups * KB * N;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const int gk = i / N;
+    const int n = i - gk * N;
+    const int g = gk / KB;
+    const int kb = gk - g * KB;
+    const uint8_t* row = src + (static_cast<size_t>(g) * N + n) * KS;
     const uint32_t lo = row[2 * kb];
     const uint32_t hi = 2 * kb + 1 < KS ? row[2 * kb + 1] : 127u;
     dst[i] = static_cast<uint16_t>(lo | (hi << 8));

@@ -54,6 +54,11 @@ moe_status_t check_cfg(const moe_config_t* c) {
   if (c->h_split != 0 && c->h_split != 1) return MOE_ERR_INVALID_ARG;
   if (c->wfmt != MOE_W_DENSE && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (c->wfmt != MOE_W_DENSE && c->h_split != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->wfmt != MOE_W_DENSE) {
+    // the scale relayout kernels index a matrix's scales with 32-bit integers
+    const int64_t big = D > F ? D : F;
+    if (int64_t(E) * big * ((big + 63) / 64) * 2 >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  }
   return MOE_OK;
 }
 
