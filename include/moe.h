@@ -272,9 +272,14 @@ MOE_API void moe_set_stage_events(void* const* starts, void* const* stops, int32
  * experts average at most 16 routed rows; otherwise single-CTA 128-row tiles for
  * gate/up and CTA-pair tiles for down),
  * 1 = single-CTA tiles, 2 = CTA-pair tiles (256 rows), 3 = decode kernel,
- * 4 = CTA pairs with the expert weights as the MMA's M operand (tokens in N).
- * Results are the same up to fp32 accumulation order.  MOE_ERR_INVALID_ARG for
- * other values. */
+ * 4 = CTA pairs with the expert weights as the MMA's M operand (tokens in N),
+ * 5 = moe_layer_forward as the two-kernel decode layer (router logits, then one
+ * persistent kernel for top-k, dispatch, both projections and the combine)
+ * wherever it applies: dense bf16 weights, T*k <= 512 routed rows averaging at
+ * most 16 per expert, E <= 256, k <= 8, hidden_size <= 8192; by size (0) it is
+ * taken for 2 <= T with T*k <= E.  Results are the same up to fp32 accumulation
+ * order (the decode layer's are reproducible call to call).  MOE_ERR_INVALID_ARG
+ * for other values. */
 MOE_API moe_status_t moe_set_expert_gemm_variant(int32_t variant);
 
 /* Number of kernels this library has launched in this process so far. */

@@ -13,6 +13,7 @@
 
 #include "grouped_gemm.cuh"
 #include "decode_gemm.cuh"
+#include "decode_layer.cuh"
 #include "grouped_gemm_pair.cuh"
 #include "grouped_gemm_pair_mx.cuh"
 #include "grouped_gemm_mx8.cuh"
@@ -207,7 +208,7 @@ static cudaError_t launch_wm_pair(const Launch& L, const CUtensorMap& w0, const 
 
 // Expert-GEMM variant (moe_set_expert_gemm_variant): 0 = by size, 1 = single-CTA
 // tiles, 2 = CTA-pair tiles, 3 = weight-stationary decode kernel, 4 = CTA pairs
-// with the weights in M.
+// with the weights in M, 5 = the two-kernel decode layer wherever it applies.
 inline std::atomic<int> g_gemm_variant{0};
 
 enum GemmKind { GK_SINGLE = 1, GK_PAIR = 2, GK_DECODE = 3, GK_WM_PAIR = 4 };
@@ -715,6 +716,99 @@ cudaError_t gather_rows(const Launch& L, const void* src, const int32_t* slot_of
   const int blocks = static_cast<int>(std::min<int64_t>((R + 7) / 8, int64_t(L.num_sms) * 8));
   pdl_launch(permute_gather_kernel, dim3(blocks), dim3(256), 0, L.stream, static_cast<const uint4*>(src), slot_of_row,
              static_cast<int>(R), k, static_cast<int>(T), row_bytes / 16, static_cast<uint4*>(dst));
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// the decode layer (decode_layer.cuh): router logits, then one persistent kernel
+// ---------------------------------------------------------------------------
+// Shapes it serves: bf16, at most kDlMaxRows routed rows and experts averaging at
+// most 16 of them (the weight-streaming regime), E <= 256 and k <= 8 (the warp top-k).
+bool decode_layer_shape(bool bf16, int64_t T, int k, int E, int D, int F) {
+  const int64_t R = T * k;
+  return bf16 && R >= 1 && R <= kDlMaxRows && R <= int64_t(16) * E && E <= kDlMaxExperts && k <= 8 &&
+         D % 8 == 0 && F % 8 == 0 && D / 8 <= kRouterMaxChunks;
+}
+
+size_t decode_layer_counter_words(int64_t T, int k, int E, int D, int F) {
+  return static_cast<size_t>(dl_counters(T, k, E, D, F).total);
+}
+
+size_t decode_layer_part_bytes() { return kDlPartFloats * sizeof(float); }
+
+// Variant 5 takes it for every shape it serves.  By size (variant 0) it is taken from two
+// tokens up to one routed row per expert on average: measured on the GPT-OSS-20B layer
+// (graph replay, 4 rotated weight copies) it beats the separate kernels at T = 2, 4, 8
+// (93 / 138 / 188 us against 100 / 159 / 201 us), ties at T = 16 and loses at T = 1 and
+// T >= 12, where its fixed hand-off latencies (dispatch, the gate/up -> down wait, the last
+// partial sums and the combine) weigh more than its balanced weight stream gains.
+bool decode_layer_selected(bool bf16, int64_t T, int k, int E, int D, int F) {
+  const int v = g_gemm_variant.load();
+  if (v == 5) return decode_layer_shape(bf16, T, k, E, D, F);
+  return v == 0 && T >= 2 && T * k <= E && decode_layer_shape(bf16, T, k, E, D, F);
+}
+
+cudaError_t decode_layer(const Launch& L, int64_t T, int D, int F, int E, int k, const void* x, const void* w_router,
+                         const void* b_router, const ExpertWeights& w, float limit, float alpha, float gate_lo,
+                         int h_halves, bool out_f32, void* y, int32_t* ids_out, float* w_out, float* logits, int* cnt,
+                         float* part, void* h, float* ys) {
+  if (T == 0) return cudaSuccess;
+  CUtensorMap wg, wu, wd;
+  cudaError_t e;
+  if ((e = make_tmap(&wg, w.w_gate, false, D, F, E, 64)) != cudaSuccess) return e;
+  if ((e = make_tmap(&wu, w.w_up, false, D, F, E, 64)) != cudaSuccess) return e;
+  if ((e = make_tmap(&wd, w.w_down, false, F, D, E, 64)) != cudaSuccess) return e;
+  const DlCounters dc = dl_counters(T, k, E, D, F);
+  const int rblocks = static_cast<int>(T) * ((E + 7) / 8);
+  const int rgrid = std::max(1, std::min(rblocks, 4 * L.num_sms));
+  pdl_launch(decode_router_kernel, dim3(rgrid), dim3(256), 0, L.stream, static_cast<const __nv_bfloat16*>(x),
+             static_cast<const __nv_bfloat16*>(w_router), static_cast<const __nv_bfloat16*>(b_router),
+             static_cast<int>(T), D, E, logits, cnt, dc.total);
+  count_launch();
+  DecLayerArgs a{};
+  a.logits = logits;
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.h = static_cast<__nv_bfloat16*>(h);
+  a.ys = ys;
+  a.y = y;
+  a.ids_out = ids_out;
+  a.w_out = w_out;
+  a.b_gate = static_cast<const __nv_bfloat16*>(w.b_gate);
+  a.b_up = static_cast<const __nv_bfloat16*>(w.b_up);
+  a.b_down = static_cast<const __nv_bfloat16*>(w.b_down);
+  a.part = part;
+  a.cnt = cnt;
+  a.off_done = dc.off_done;
+  a.off_gu = dc.off_gu;
+  a.off_dn = dc.off_dn;
+  a.off_cb = dc.off_cb;
+  a.T = static_cast<int>(T);
+  a.k = k;
+  a.E = E;
+  a.D = D;
+  a.F = F;
+  a.h_halves = h_halves;
+  a.out_f32 = out_f32 ? 1 : 0;
+  a.limit = limit;
+  a.alpha = alpha;
+  a.gate_lo = gate_lo;
+  a.wait_limit_ns = L.wait_limit_ns;
+  constexpr int smem = DlLayout::smem_bytes;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static std::mutex mu;
+  static uint64_t configured = 0;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (dev >= 64 || !((configured >> dev) & 1u)) {
+      e = cudaFuncSetAttribute(decode_layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) configured |= uint64_t(1) << dev;
+    }
+  }
+  const int grid = std::min(L.num_sms, kDlMaxCtas);
+  pdl_launch(decode_layer_kernel, dim3(grid), dim3(kDlThreads), smem, L.stream, wg, wu, wd, a);
   count_launch();
   return cudaGetLastError();
 }

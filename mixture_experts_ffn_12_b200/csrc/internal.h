@@ -99,6 +99,20 @@ cudaError_t expert_down_mxfp4(const Launch& L, int64_t R, int D, int F, int E, c
                               const int32_t* expert_off, const ExpertWeights& w, const uint8_t* s_down2,
                               const int32_t* slot_of_row, const float* topk_w, void* out);
 
+// The whole layer for a few tokens (bf16; decode_layer_shape): router logits into
+// `logits` [T, E], then one persistent kernel for top-k, dispatch, both projections and
+// the combine.  Scratch: cnt (decode_layer_counter_words ints), part
+// (decode_layer_part_bytes), h [R, h_halves * F], ys [R, D] fp32.  x and the rows of h are
+// read with 16-byte copies (x 16-byte aligned).  ids_out / w_out [T, k] may be null.
+bool decode_layer_shape(bool bf16, int64_t T, int k, int E, int D, int F);
+bool decode_layer_selected(bool bf16, int64_t T, int k, int E, int D, int F);
+size_t decode_layer_counter_words(int64_t T, int k, int E, int D, int F);
+size_t decode_layer_part_bytes();
+cudaError_t decode_layer(const Launch& L, int64_t T, int D, int F, int E, int k, const void* x, const void* w_router,
+                         const void* b_router, const ExpertWeights& w, float limit, float alpha, float gate_lo,
+                         int h_halves, bool out_f32, void* y, int32_t* ids_out, float* w_out, float* logits, int* cnt,
+                         float* part, void* h, float* ys);
+
 cudaError_t read_and_clear_device_error(int* bits);
 
 }  // namespace moe

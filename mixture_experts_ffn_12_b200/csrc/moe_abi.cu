@@ -97,7 +97,16 @@ size_t ffn_ws_bytes(const moe_config_t* c, int64_t) { return c->wfmt == MOE_W_MX
 
 struct Layout {
   size_t ids, w, off, ros, sor, pscr, xperm, h, rpart, ys, ffn, total;
+  bool dl;                        // the decode layer's regions follow
+  size_t dlog, dcnt, dpart, dys;  // its router logits, counters, partial sums, weighted rows
 };
+
+// Whether a layer of T tokens can run as the two-kernel decode layer (dense bf16 weights).
+bool decode_layer_shape(const moe_config_t* c, int64_t T) {
+  return c->wfmt == MOE_W_DENSE &&
+         moe::decode_layer_shape(c->dtype == MOE_BF16, T, c->num_experts_per_tok, c->num_local_experts,
+                                 c->hidden_size, c->intermediate_size);
+}
 
 Layout layout(const moe_config_t* c, int64_t T) {
   const size_t R = size_t(T) * c->num_experts_per_tok, es = elem_size(c);
@@ -123,6 +132,15 @@ Layout layout(const moe_config_t* c, int64_t T) {
   L.h = take(h_bytes > rpart_bytes ? h_bytes : rpart_bytes);
   L.rpart = L.h;
   L.ffn = take(ffn_ws_bytes(c, T));
+  L.dl = decode_layer_shape(c, T);
+  if (L.dl) {
+    // the decode layer writes the weighted rows while other CTAs still read x_perm: own region
+    L.dlog = take(size_t(T) * c->num_local_experts * 4);
+    L.dcnt = take(moe::decode_layer_counter_words(T, c->num_experts_per_tok, c->num_local_experts, c->hidden_size,
+                                                  c->intermediate_size) * 4);
+    L.dpart = take(moe::decode_layer_part_bytes());
+    L.dys = take(R * c->hidden_size * 4);
+  }
   L.total = o;
   return L;
 }
@@ -576,6 +594,19 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x
   const bool bf16 = cfg->dtype == MOE_BF16;
   const int D = cfg->hidden_size, E = cfg->num_local_experts, k = cfg->num_experts_per_tok;
 
+  if (LY.dl && moe::decode_layer_selected(bf16, T, k, E, D, cfg->intermediate_size)) {
+    stage_mark(ST_ROUTER, true, L.stream);
+    stage_mark(ST_ROUTER, false, L.stream);
+    stage_mark(ST_GATEUP, true, L.stream);
+    const moe_status_t st = cuda_status(moe::decode_layer(
+        L, T, D, cfg->intermediate_size, E, k, x, w_router, b_router, to_internal(weights), cfg->swiglu_limit,
+        cfg->swiglu_alpha, 0.0f, h_halves(cfg), !out_bf16(cfg), y, topk_ids_out, topk_w_out,
+        reinterpret_cast<float*>(base + LY.dlog), reinterpret_cast<int*>(base + LY.dcnt),
+        reinterpret_cast<float*>(base + LY.dpart), h, reinterpret_cast<float*>(base + LY.dys)));
+    stage_mark(ST_GATEUP, false, L.stream);
+    return st;
+  }
+
   stage_mark(ST_ROUTER, true, L.stream);
   if (moe::router_topk(L, bf16, T, D, E, k, x, w_router, b_router, ids, w,
                        reinterpret_cast<float*>(base + LY.rpart)) != cudaSuccess)
@@ -623,7 +654,7 @@ void moe_set_stage_events(void* const* starts, void* const* stops, int32_t n) {
 uint64_t moe_launch_count(void) { return moe::g_launches.load(); }
 
 moe_status_t moe_set_expert_gemm_variant(int32_t variant) {
-  if (variant < 0 || variant > 4) return MOE_ERR_INVALID_ARG;
+  if (variant < 0 || variant > 5) return MOE_ERR_INVALID_ARG;
   moe::g_gemm_variant.store(variant);
   return MOE_OK;
 }
