@@ -41,7 +41,7 @@ constexpr int kDlMaxExperts = 256;
 constexpr int kDlMaxCtas = 160;      // grid = min(SMs, this); sizes the partial buffers
 constexpr int kDlThreads = 224;     // producer, MMA, 4 epilogue warps, gather warp
 constexpr int kDlWarps = kDlThreads / 32;
-constexpr int kDlGatherLag = 3;    // stages between a token copy's issue and the wait for it
+constexpr int kDlGatherLag = 6;    // stages between a token copy's issue and the wait for it
 // weight tiles issued ahead of the token copies: a deeper burst while the gather warp waits
 // for h queues the hand-off's own small messages (counters, partial sums) behind it
 constexpr int kDlHoldAhead = 2;
