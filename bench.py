@@ -413,6 +413,13 @@ def decode_sweep(api, moe, spec, layer, dev, stream, steps, copies=4):
             moe(x, topk_ids=ids)
         torch.cuda.synchronize()
         touched = int(torch.unique(ids).numel())
+        # kernels one layer call launches: 2 = the two-kernel decode layer, more = separate kernels
+        from mixture_experts_ffn_12_b200 import _lib
+        lib = _lib.load()
+        n0 = lib.moe_launch_count()
+        moe(x, topk_ids=ids)
+        launches = int(lib.moe_launch_count() - n0)
+        torch.cuda.synchronize()
         # CUDA-graph replay of the same launches (host launch overhead removed), one graph per copy
         replays = [lyr.graphed(x, topk_ids=torch.empty_like(ids))[0] for lyr in layers]
         for i in range(3 * copies):
@@ -427,7 +434,9 @@ def decode_sweep(api, moe, spec, layer, dev, stream, steps, copies=4):
         us = 1e3 * a.elapsed_time(b) / n
         nbytes = touched * 3 * spec.D * spec.F * esz + spec.E * spec.D * esz
         gbs = nbytes / (us * 1e-6) / 1e9
-        out[f"T{T}"] = {"us_per_step": us, "experts_touched": touched, "weight_bytes": nbytes, "GB/s": gbs,
+        out[f"T{T}"] = {"us_per_step": us, "launches_per_step": launches,
+                        "path": "two-kernel decode layer" if launches == 2 else "separate kernels",
+                        "experts_touched": touched, "weight_bytes": nbytes, "GB/s": gbs,
                         "hbm_frac": gbs / peaks["hbm_gbs"], "tokens/s": T / (us * 1e-6)}
         del replays
     del layers
