@@ -462,7 +462,8 @@ def set_expert_gemm_variant(variant: int) -> None:
     """Expert-GEMM kernel choice for bf16 dense weights: 0 = by size (the default), 1 = single-CTA
     128-row tiles, 2 = CTA-pair 256-row tiles, 3 = the weight-stationary decode kernel,
     4 = CTA pairs with the weights in M, 5 = layer_forward as the two-kernel decode layer
-    wherever it applies.  Process-wide; MXFP4 layers ignore it."""
+    wherever it applies, 6 = by size with the layer's gate/up rows gathered from x (TMA gather4)
+    rather than read from x_perm.  Process-wide; MXFP4 layers ignore it."""
     _check(_lib.load().moe_set_expert_gemm_variant(variant), "moe_set_expert_gemm_variant")
 
 

@@ -166,6 +166,18 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
       : "memory");
 }
 
+// Four rows of a 2-D tensor map (box: one row of box[0] elements) at column c0 into
+// shared memory: rows r0..r3 land as four consecutive rows of the destination, which is
+// laid out (and 128-byte swizzled, by shared-memory address) as a box of four rows would be.
+__device__ __forceinline__ void tma_gather4_2d(void* dst, const void* tmap, uint64_t* bar, int c0, int r0, int r1,
+                                               int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
 // --------------------------------------------------------------------------
 // tcgen05 (cta_group::1)
 // --------------------------------------------------------------------------

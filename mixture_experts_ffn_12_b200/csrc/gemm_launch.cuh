@@ -208,7 +208,8 @@ static cudaError_t launch_wm_pair(const Launch& L, const CUtensorMap& w0, const 
 
 // Expert-GEMM variant (moe_set_expert_gemm_variant): 0 = by size, 1 = single-CTA
 // tiles, 2 = CTA-pair tiles, 3 = weight-stationary decode kernel, 4 = CTA pairs
-// with the weights in M, 5 = the two-kernel decode layer wherever it applies.
+// with the weights in M, 5 = the two-kernel decode layer wherever it applies,
+// 6 = by size, except that the layer's gate/up rows are gathered from x (TMA gather4).
 inline std::atomic<int> g_gemm_variant{0};
 
 enum GemmKind { GK_SINGLE = 1, GK_PAIR = 2, GK_DECODE = 3, GK_WM_PAIR = 4 };
@@ -402,10 +403,19 @@ cudaError_t expert_down_mxfp4(const Launch& L, int64_t R, int D, int F, int E, c
   return launch_pair_mx<kTNHalf, EPI_BIAS, kMxStages>(L, ta, pd, pd, sd, sd, a, ptiles);
 }
 
+// Whether the single-CTA gate/up kernel takes its A rows from x by TMA gather4 (so the
+// layer needs no x_perm): only with expert-GEMM variant 6.  Correct (bit-identical to the
+// x_perm form) but slower: a 128-row A tile takes 32 gather4 loads per 64-wide K block,
+// and on the GPT-OSS-20B prefill layer gate/up ran 1.38-1.41 ms against 0.50 ms.
+bool gateup_gathers(bool bf16, int64_t R, int E) {
+  return bf16 && g_gemm_variant.load() == 6 && gemm_kind(R, E) == GK_SINGLE;
+}
+
 cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,
                           const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h,
-                          float gate_lo, int h_halves) {
+                          float gate_lo, int h_halves, const GateupGather* gather) {
   if (R == 0) return cudaSuccess;
+  if (gather != nullptr && !gateup_gathers(bf16, R, E)) return cudaErrorInvalidValue;
   if (h_halves == 2 && (!bf16 || gemm_kind(R, E) == GK_WM_PAIR)) return cudaErrorNotSupported;
   if (!bf16) {
     GemmArgs a = base_args(L);
@@ -429,10 +439,18 @@ cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, i
   }
   CUtensorMap ta, tg, tu;
   cudaError_t e;
-  if ((e = make_tmap(&ta, x_perm, !bf16, D, R, 0, kBM)) != cudaSuccess) return e;
+  // gathering: A is x [T, D] with one-row boxes, read four rows per gather4
+  if (gather != nullptr) e = make_tmap(&ta, gather->x, false, D, gather->T, 0, 1);
+  else e = make_tmap(&ta, x_perm, !bf16, D, R, 0, kBM);
+  if (e != cudaSuccess) return e;
   if ((e = make_tmap(&tg, w.w_gate, !bf16, D, F, E, kTNGateUp)) != cudaSuccess) return e;
   if ((e = make_tmap(&tu, w.w_up, !bf16, D, F, E, kTNGateUp)) != cudaSuccess) return e;
   GemmArgs a = base_args(L);
+  if (gather != nullptr) {
+    a.gather_slots = gather->slot_of_row;
+    a.gather_k = gather->k;
+    a.gather_rows = static_cast<int>(gather->T);
+  }
   a.group_off = expert_off;
   a.num_groups = E;
   a.m_total = static_cast<int>(R);

@@ -70,6 +70,9 @@ struct GemmArgs {
   const uint8_t* scale1;
   int k_splits;                // EPI_PARTIAL: K ranges; column block index = K range
   float* partial;              // EPI_PARTIAL: [k_splits, n_out, m_total] fp32
+  const int32_t* gather_slots; // non-null (EPI_SWIGLU, bf16): A row r is row gather_slots[r] / gather_k of
+  int gather_k;                //   the tensor map's matrix (x), loaded four rows at a time with TMA
+  int gather_rows;             //   gather4; rows of that matrix (clamp for rows past a group's end)
   int h_halves;                // 2: h is kept as two bf16 halves per row, [R, 2, F] (h = hi + lo):
                                // EPI_SWIGLU writes hi = bf16(h) and lo = bf16(h - hi); the down
                                // GEMM reads h through a 3-D tensor map {F, 2, R} and sums over
@@ -377,7 +380,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = tile_off[G] * NT;
 
-  if (warp == 0) {
+  if (warp == 0 && EPI == EPI_SWIGLU && !kTF32 && args.gather_slots != nullptr) {
+    // ------------------------------------------------------------ TMA producer, A rows gathered
+    // Lane j loads A rows 4j .. 4j + 3 of every stage with one gather4 from x (the row of
+    // each permuted row's token); lane 0 waits for the slot, arms the barrier and loads B.
+    const uint32_t tx_bytes = LY::A_BYTES + static_cast<uint32_t>(TN * NB) * kRowBytes;
+    int s = 0;
+    uint32_t ph = 0, issued = 0, issued_par = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+      const TileInfo ti = decode_tile(i, tile_off, goff, G, NT, TN);
+      int src[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int row = ti.m0 + 4 * lane + q;
+        int t = 0;
+        if (row < ti.m_end) {
+          t = __ldg(args.gather_slots + row) / args.gather_k;
+          if (t < 0 || t >= args.gather_rows) { flag_error(DEVERR_BOUNDS); t = 0; }
+        }
+        src[q] = t;   // rows past the group read row 0; their outputs are never written
+      }
+      for (int kb = 0; kb < KB; ++kb) {
+        bool got = true;
+        if (lane == 0) {
+          got = mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim);
+          if (got) mbar_arrive_expect_tx(&full[s], tx_bytes);
+        }
+        if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) { ok = false; break; }
+        uint8_t* sa = smem + s * LY::STAGE_BYTES;
+        tma_gather4_2d(sa + 4 * lane * kRowBytes, &tmA, &full[s], kb * BK, src[0], src[1], src[2], src[3]);
+        if (lane == 0) {
+          uint8_t* sb = sa + LY::A_BYTES;
+          tma_load_3d(sb, &tmB0, &full[s], kb * BK, ti.n0, ti.g);
+          if (NB == 2) tma_load_3d(sb + TN * kRowBytes, &tmB1, &full[s], kb * BK, ti.n0, ti.g);
+        }
+        issued |= 1u << s;
+        issued_par = (issued_par & ~(1u << s)) | (ph << s);
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      }
+    }
+    if (lane == 0) {
+      if (!ok) {
+        *abort_flag = 1;
+        flag_error(DEVERR_TIMEOUT);
+      }
+      for (int q = 0; q < STAGES; ++q)
+        if ((issued >> q) & 1u)
+          if (!mbar_wait(&full[q], (issued_par >> q) & 1u, never_flag, kDrainLimitNs)) flag_error(DEVERR_TIMEOUT);
+    }
+    __syncwarp();
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const int mma_n = (EPI == EPI_TOPK || EPI == EPI_PARTIAL) ? args.mma_n : TN * NB;

@@ -47,9 +47,19 @@ struct ExpertWeights {
 // alpha = 1 gives SiLU(g) * u.  h_halves = 2 (bf16 only): h is [R, 2, F], the bf16 rounding
 // of h and the bf16 rounding of what that dropped (cudaErrorNotSupported for the fp32
 // kernels and the weights-in-M pair kernel).
+// gather (the layer only): A row r is x[slot_of_row[r] / k] (x [T, D] bf16), read by TMA
+// gather4 instead of from x_perm, which is then not read (may be null); only where
+// gateup_gathers() holds.
+struct GateupGather {
+  const void* x;
+  const int32_t* slot_of_row;
+  int k;
+  int64_t T;
+};
+bool gateup_gathers(bool bf16, int64_t R, int E);
 cudaError_t expert_gateup(const Launch& L, bool bf16, int64_t R, int D, int F, int E, const void* x_perm,
                           const int32_t* expert_off, const ExpertWeights& w, float limit, float alpha, void* h,
-                          float gate_lo = 0.0f, int h_halves = 1);
+                          float gate_lo = 0.0f, int h_halves = 1, const GateupGather* gather = nullptr);
 
 // Down projection.  If slot_of_row == nullptr: out[r] = h[r] W_d^T + b_d (permuted order, dtype);
 // else out[slot_of_row[r]] = topk_w[slot] * (h[r] W_d^T + b_d) (slot order, fp32).

@@ -238,7 +238,8 @@ moe::ExpertWeights to_internal(const moe_expert_weights_t* w) {
 // gate/up then down (into y_perm, or weighted into slot order when slot_of_row != null)
 moe_status_t run_experts(const moe_config_t* c, const Launch& L, int64_t T, const void* x_perm,
                          const int32_t* eoff, const moe_expert_weights_t* wts, void* h, void* out,
-                         const int32_t* slot_of_row, const float* topk_w, void* ffn_ws) {
+                         const int32_t* slot_of_row, const float* topk_w, void* ffn_ws,
+                         const moe::GateupGather* gather = nullptr) {
   const bool bf16 = c->dtype == MOE_BF16;
   const int D = c->hidden_size, F = c->intermediate_size, E = c->num_local_experts;
   const int64_t R = T * c->num_experts_per_tok;
@@ -260,8 +261,8 @@ moe_status_t run_experts(const moe_config_t* c, const Launch& L, int64_t T, cons
     return st;
   }
   const int hh = h_halves(c);
-  if (moe::expert_gateup(L, bf16, R, D, F, E, x_perm, eoff, w, c->swiglu_limit, c->swiglu_alpha, h, 0.0f, hh) !=
-      cudaSuccess)
+  if (moe::expert_gateup(L, bf16, R, D, F, E, x_perm, eoff, w, c->swiglu_limit, c->swiglu_alpha, h, 0.0f, hh,
+                         gather) != cudaSuccess)
     return MOE_ERR_CUDA;
   stage_mark(ST_GATEUP, false, L.stream);
   stage_mark(ST_DOWN, true, L.stream);
@@ -612,10 +613,16 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, int64_t T, const void* x
                        reinterpret_cast<float*>(base + LY.rpart)) != cudaSuccess)
     return MOE_ERR_CUDA;
   stage_mark(ST_ROUTER, false, L.stream);
+  // with expert-GEMM variant 6 the single-CTA gate/up kernel gathers its A rows from x
+  // (TMA gather4): the dispatch then builds the maps only, with no x_perm copy
+  const bool gather = cfg->wfmt == MOE_W_DENSE && moe::gateup_gathers(bf16, T * k, E);
+  const moe::GateupGather gx{x, sor, k, T};
   stage_mark(ST_DISPATCH, true, L.stream);
-  if (moe::permute(L, bf16, T, D, E, k, ids, x, eoff, ros, sor, xperm, pscr) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::permute(L, bf16, T, D, E, k, ids, gather ? nullptr : x, eoff, ros, sor, gather ? nullptr : xperm, pscr) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
   stage_mark(ST_DISPATCH, false, L.stream);
-  s = run_experts(cfg, L, T, xperm, eoff, weights, h, ys, sor, w, ffn);
+  s = run_experts(cfg, L, T, xperm, eoff, weights, h, ys, sor, w, ffn, gather ? &gx : nullptr);
   if (s != MOE_OK) return s;
   stage_mark(ST_COMBINE, true, L.stream);
   s = cuda_status(moe::combine_slots(L, out_bf16(cfg), T, D, k, ys, y));
@@ -654,7 +661,7 @@ void moe_set_stage_events(void* const* starts, void* const* stops, int32_t n) {
 uint64_t moe_launch_count(void) { return moe::g_launches.load(); }
 
 moe_status_t moe_set_expert_gemm_variant(int32_t variant) {
-  if (variant < 0 || variant > 5) return MOE_ERR_INVALID_ARG;
+  if (variant < 0 || variant > 6) return MOE_ERR_INVALID_ARG;
   moe::g_gemm_variant.store(variant);
   return MOE_OK;
 }
