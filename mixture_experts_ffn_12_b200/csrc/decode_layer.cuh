@@ -267,61 +267,9 @@ __global__ void __launch_bounds__(kDlThreads, 1)
       }
       warp_topk_softmax(v, lane, E, k, ids_s + t * k, w_s + t * k);
     }
-  } else for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    const float* lg = a.logits + static_cast<size_t>(t) * E;
-    float tv[8];
-    int ti[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      tv[j] = -INFINITY;
-      ti[j] = 0x7fffffff;
-    }
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      float v32[32];
-      if ((E & 3) == 0) {
-#pragma unroll
-        for (int u = 0; u < 32; u += 4) {
-          float4 f4 = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-          if (e0 + u < E) f4 = __ldcg(reinterpret_cast<const float4*>(lg + e0 + u));
-          v32[u] = f4.x;
-          v32[u + 1] = f4.y;
-          v32[u + 2] = f4.z;
-          v32[u + 3] = f4.w;
-        }
-      } else {
-#pragma unroll
-        for (int u = 0; u < 32; ++u) v32[u] = e0 + u < E ? __ldcg(lg + e0 + u) : -INFINITY;
-      }
-#pragma unroll
-      for (int u = 0; u < 32; ++u) {
-        float cv = v32[u];
-        int ci = e0 + u;
-        if (ci >= E || !(cv > tv[7])) continue;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const bool gt = cv > tv[q];
-          const float tq = tv[q];
-          const int iq = ti[q];
-          tv[q] = gt ? cv : tq;
-          ti[q] = gt ? ci : iq;
-          cv = gt ? tq : cv;
-          ci = gt ? iq : ci;
-        }
-      }
-    }
-    float z = 0.0f, ex[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      ex[j] = j < k ? expf(tv[j] - tv[0]) : 0.0f;
-      z += ex[j];
-    }
-    const float inv = 1.0f / z;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j < k) {
-        ids_s[t * k + j] = ti[j];
-        w_s[t * k + j] = ex[j] * inv;
-      }
+  } else {
+    for (int t = threadIdx.x; t < T; t += blockDim.x)
+      thread_topk_softmax(a.logits + static_cast<size_t>(t) * E, E, k, ids_s + t * k, w_s + t * k);
   }
   tc_fence_before();
   __syncthreads();
