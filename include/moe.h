@@ -277,8 +277,9 @@ MOE_API void moe_set_stage_events(void* const* starts, void* const* stops, int32
  * persistent kernel for top-k, dispatch, both projections and the combine)
  * wherever it applies: dense bf16 weights, T*k <= 512 routed rows averaging at
  * most 16 per expert, E <= 256, k <= 8, hidden_size <= 8192; by size (0) it is
- * taken for 2 <= T with T*k <= E; 6 = as 0, except that moe_layer_forward's
- * single-CTA gate/up kernel gathers its rows from x with TMA gather4 instead of
+ * taken for 2 <= T with T*k <= E; 6 = as 0 (but never the decode layer), except
+ * that moe_layer_forward's single-CTA gate/up kernel gathers its rows from x with
+ * TMA gather4 instead of
  * reading a dispatched copy (x_perm), which is then not written (same results bit
  * for bit; slower).  Results are the same up to fp32 accumulation order (the
  * decode layer's are reproducible call to call).  MOE_ERR_INVALID_ARG for other
