@@ -281,7 +281,10 @@ MOE_API void moe_set_stage_events(void* const* starts, void* const* stops, int32
  * that moe_layer_forward's single-CTA gate/up kernel gathers its rows from x with
  * TMA gather4 instead of
  * reading a dispatched copy (x_perm), which is then not written (same results bit
- * for bit; slower).  Results are the same up to fp32 accumulation order (the
+ * for bit; slower); 7 = as 6 without the gather, and the MOE_W_MXFP4_A8 GEMMs
+ * widen every stage of E2M1 weights in their converter warps instead of loading
+ * whole 128-code K blocks through TMA's 4-bit unpacking type (same results bit for
+ * bit).  Results are the same up to fp32 accumulation order (the
  * decode layer's are reproducible call to call).  MOE_ERR_INVALID_ARG for other
  * values. */
 MOE_API moe_status_t moe_set_expert_gemm_variant(int32_t variant);

@@ -463,7 +463,9 @@ def set_expert_gemm_variant(variant: int) -> None:
     128-row tiles, 2 = CTA-pair 256-row tiles, 3 = the weight-stationary decode kernel,
     4 = CTA pairs with the weights in M, 5 = layer_forward as the two-kernel decode layer
     wherever it applies, 6 = by size with the layer's gate/up rows gathered from x (TMA gather4)
-    rather than read from x_perm.  Process-wide; MXFP4 layers ignore it."""
+    rather than read from x_perm, 7 = by size, with the MXFP4 x MXFP8 GEMMs widening every E2M1
+    stage in their converter warps (no TMA 4-bit unpacking).  Process-wide; other MXFP4 layers
+    ignore it."""
     _check(_lib.load().moe_set_expert_gemm_variant(variant), "moe_set_expert_gemm_variant")
 
 

@@ -209,7 +209,8 @@ static cudaError_t launch_wm_pair(const Launch& L, const CUtensorMap& w0, const 
 // Expert-GEMM variant (moe_set_expert_gemm_variant): 0 = by size, 1 = single-CTA
 // tiles, 2 = CTA-pair tiles, 3 = weight-stationary decode kernel, 4 = CTA pairs
 // with the weights in M, 5 = the two-kernel decode layer wherever it applies,
-// 6 = by size, except that the layer's gate/up rows are gathered from x (TMA gather4).
+// 6 = by size, except that the layer's gate/up rows are gathered from x (TMA gather4),
+// 7 = by size, and the MXFP4 x MXFP8 GEMMs widen every E2M1 stage in their converter warps.
 inline std::atomic<int> g_gemm_variant{0};
 
 enum GemmKind { GK_SINGLE = 1, GK_PAIR = 2, GK_DECODE = 3, GK_WM_PAIR = 4 };
@@ -618,9 +619,31 @@ static cudaError_t make_tmap_e2m1(CUtensorMap* m, const void* ptr, uint64_t K, u
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// The same weights through TMA's 4-bit unpacking type: each 16 codes land in 16 bytes of
+// shared memory (the upper 8 unused), 128-byte swizzle -- the tile the f8f6f4 MMA reads.
+// The type describes rows in whole 128-code blocks: dims {K rounded down to 128, N, G};
+// boxes of 128 codes x box_rows.  Its strides and base need 32-byte alignment.
+// (Expert-GEMM variant 7 turns the unpacking off: every stage is widened by the converters.)
+static bool e2m1_unpack_ok(const void* ptr, uint64_t K) {
+  return g_gemm_variant.load() != 7 && K >= 128 && (K / 2) % 32 == 0 && (reinterpret_cast<uintptr_t>(ptr) & 31u) == 0;
+}
+static cudaError_t make_tmap_e2m1_unpack(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t N, uint64_t G,
+                                         uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {K / kMx8BK * kMx8BK, N, G};
+  const cuuint64_t strides[2] = {K / 2, (K / 2) * N};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kMx8BK), box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int EPI, int TN, int NB, int STAGES>
 static cudaError_t launch_mx8(const Launch& L, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                              const Mx8Args& args, int64_t max_tiles) {
+                              const CUtensorMap& u0, const CUtensorMap& u1, const Mx8Args& args, int64_t max_tiles) {
   if (max_tiles <= 0) return cudaSuccess;
   auto kern = grouped_gemm_mx8_kernel<EPI, TN, NB, STAGES>;
   constexpr int smem = Mx8Layout<TN, NB>::smem_bytes(STAGES);
@@ -638,7 +661,7 @@ static cudaError_t launch_mx8(const Launch& L, const CUtensorMap& a, const CUten
     }
   }
   const int grid = static_cast<int>(std::min<int64_t>(max_tiles, L.num_sms));
-  pdl_launch(kern, dim3(grid), dim3(kMx8Threads), smem, L.stream, a, b0, b1, args);
+  pdl_launch(kern, dim3(grid), dim3(kMx8Threads), smem, L.stream, a, b0, b1, u0, u1, args);
   count_launch();
   return cudaGetLastError();
 }
@@ -696,8 +719,14 @@ cudaError_t expert_gateup_mx8(const Launch& L, int64_t R, int D, int F, int E, c
   a.sfh = sfh;
   a.sfs_h = mx8_sf_stride(F);
   a.wait_limit_ns = L.wait_limit_ns;
+  CUtensorMap ug = tg, uu = tu;
+  if (e2m1_unpack_ok(w.w_gate, D) && e2m1_unpack_ok(w.w_up, D)) {
+    if ((e = make_tmap_e2m1_unpack(&ug, w.w_gate, D, F, E, kMx8TNGateUp)) != cudaSuccess) return e;
+    if ((e = make_tmap_e2m1_unpack(&uu, w.w_up, D, F, E, kMx8TNGateUp)) != cudaSuccess) return e;
+    a.kb_unpacked = D / kMx8BK;
+  }
   const int64_t tiles = max_row_blocks(R, E) * ((F + kMx8TNGateUp - 1) / kMx8TNGateUp);
-  return launch_mx8<EPI_SWIGLU, kMx8TNGateUp, 2, kMx8StagesGateUp>(L, ta, tg, tu, a, tiles);
+  return launch_mx8<EPI_SWIGLU, kMx8TNGateUp, 2, kMx8StagesGateUp>(L, ta, tg, tu, ug, uu, a, tiles);
 }
 
 cudaError_t expert_down_mx8(const Launch& L, int64_t R, int D, int F, int E, const uint8_t* hq, const uint8_t* sfh,
@@ -723,8 +752,13 @@ cudaError_t expert_down_mx8(const Launch& L, int64_t R, int D, int F, int E, con
   a.slot_of_row = slot_of_row;
   a.topk_w = topk_w;
   a.wait_limit_ns = L.wait_limit_ns;
+  CUtensorMap ud = td;
+  if (e2m1_unpack_ok(w.w_down, F)) {
+    if ((e = make_tmap_e2m1_unpack(&ud, w.w_down, F, D, E, kMx8TNDown)) != cudaSuccess) return e;
+    a.kb_unpacked = F / kMx8BK;
+  }
   const int64_t tiles = max_row_blocks(R, E) * ((D + kMx8TNDown - 1) / kMx8TNDown);
-  return launch_mx8<EPI_BIAS_WSCATTER, kMx8TNDown, 1, kMx8StagesDown>(L, ta, td, td, a, tiles);
+  return launch_mx8<EPI_BIAS_WSCATTER, kMx8TNDown, 1, kMx8StagesDown>(L, ta, td, td, ud, ud, a, tiles);
 }
 
 // x_perm-style row gather of byte rows (row_bytes a multiple of 16): dst[r] = src[slot_of_row[r] / k].

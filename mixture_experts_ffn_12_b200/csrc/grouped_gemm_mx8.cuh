@@ -15,12 +15,15 @@
 // Operands in shared memory (128-byte swizzle, K-major, 128 K elements a stage):
 //   A  E4M3 rows by TMA (uint8 tensor map), 128 rows x 128 B.
 //   B  the f8f6f4 MMA reads 4-bit operands with each 16 codes (8 B) in 16 B of
-//      shared memory, the upper 8 B unused.  The packed rows (64 B per 128 codes)
-//      arrive by a plain byte TMA in a staging area; four converter warps widen
-//      every 8 B to 16 B (zeros above) into the 128-byte-swizzled tile the MMA
-//      reads -- byte moves only, any K that is a multiple of 32.  (TMA's own
-//      unpacking type needs row lengths and start coordinates in 128-code units,
-//      which K = 2880 is not.)
+//      shared memory, the upper 8 B unused.  Whole 128-code K blocks come by TMA
+//      with its 4-bit unpacking type (16U4_ALIGN16B), which writes exactly that
+//      layout into the 128-byte-swizzled tile; the unpacking type wants the rows
+//      described in whole 128-code blocks, so a last partial block (K = 2880 =
+//      22.5 x 128) and weights the type cannot describe (K / 2 not a multiple of
+//      32 bytes, or a base not 32-byte aligned) arrive packed (64 B per 128 codes)
+//      by a plain byte TMA in a staging area, and four converter warps widen every
+//      8 B to 16 B (zeros above) into the tile -- byte moves only, any K that is a
+//      multiple of 32.
 //   SF the E8M0 scales, loaded by a warp of their own with 32-bit loads (four
 //      K blocks = one stage per load) from row-major copies padded to SFS bytes
 //      a row, stored into the 512-byte chunks tcgen05.cp copies to TMEM: byte
@@ -256,6 +259,7 @@ struct Mx8Args {
   const int32_t* slot_of_row;
   const float* topk_w;
   unsigned long long wait_limit_ns;
+  int kb_unpacked;            // K blocks [0, kb_unpacked) come through the unpacking maps
 };
 
 // ---------------------------------------------------------------------------
@@ -343,11 +347,13 @@ __device__ __forceinline__ void mx8_epi_wscatter(uint32_t tbase, int row, bool r
 // the kernel
 // ---------------------------------------------------------------------------
 // tmA: E4M3 activations [m_total, K]; tmB0 / tmB1: packed E2M1 weights [G, n_out, K/2] bytes,
-// boxes of 64 B (128 codes) x TN rows.
+// boxes of 64 B (128 codes) x TN rows; tmU0 / tmU1: the same weights through the 4-bit
+// unpacking type, boxes of 128 codes x TN rows (used for K blocks below kb_unpacked).
 template <int EPI, int TN, int NB, int STAGES>
 __global__ void __launch_bounds__(kMx8Threads, 1)
     grouped_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                            const __grid_constant__ CUtensorMap tmB1, const Mx8Args args) {
+                            const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmU0,
+                            const __grid_constant__ CUtensorMap tmU1, const Mx8Args args) {
   pdl_enter();
   using LY = Mx8Layout<TN, NB>;
   constexpr int N = LY::N;
@@ -427,6 +433,10 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB0);
       if (NB == 2) tma_prefetch_desc(&tmB1);
+      if (args.kb_unpacked > 0) {
+        tma_prefetch_desc(&tmU0);
+        if (NB == 2) tma_prefetch_desc(&tmU1);
+      }
     }
   } else if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -441,6 +451,7 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // an unpacked box counts the packed bytes it reads, as a packed box does
       const uint32_t tx_bytes = LY::A_BYTES + LY::P_BYTES;
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_par = 0;
@@ -451,8 +462,13 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], tx_bytes);
           tma_load_2d(stage_a(s), &tmA, &full[s], kb * kMx8BK, ti.m0);
-          tma_load_3d(stage_p(s), &tmB0, &full[s], kb * (kMx8BK / 2), ti.n0, ti.g);
-          if (NB == 2) tma_load_3d(stage_p(s) + TN * (kMx8BK / 2), &tmB1, &full[s], kb * (kMx8BK / 2), ti.n0, ti.g);
+          if (kb < args.kb_unpacked) {
+            tma_load_3d(stage_b(s), &tmU0, &full[s], kb * kMx8BK, ti.n0, ti.g);
+            if (NB == 2) tma_load_3d(stage_b(s) + TN * kMx8BK, &tmU1, &full[s], kb * kMx8BK, ti.n0, ti.g);
+          } else {
+            tma_load_3d(stage_p(s), &tmB0, &full[s], kb * (kMx8BK / 2), ti.n0, ti.g);
+            if (NB == 2) tma_load_3d(stage_p(s) + TN * (kMx8BK / 2), &tmB1, &full[s], kb * (kMx8BK / 2), ti.n0, ti.g);
+          }
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -479,21 +495,23 @@ __global__ void __launch_bounds__(kMx8Threads, 1)
     for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
       for (int kb = 0; kb < KB; ++kb) {
         if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim))) { ok = false; break; }
-        const uint8_t* src = stage_p(s);
-        uint8_t* dst = stage_b(s);
-        uint2 v[PER];
+        if (kb >= args.kb_unpacked) {   // an unpacked stage is already in place
+          const uint8_t* src = stage_p(s);
+          uint8_t* dst = stage_b(s);
+          uint2 v[PER];
 #pragma unroll
-        for (int j = 0; j < PER; ++j) {
-          const int q = ct + j * 32 * kMx8ConvWarps;
-          v[j] = *reinterpret_cast<const uint2*>(src + 8 * q);
-        }
+          for (int j = 0; j < PER; ++j) {
+            const int q = ct + j * 32 * kMx8ConvWarps;
+            v[j] = *reinterpret_cast<const uint2*>(src + 8 * q);
+          }
 #pragma unroll
-        for (int j = 0; j < PER; ++j) {
-          const int q = ct + j * 32 * kMx8ConvWarps;
-          const int r = q >> 3, c = q & 7;
-          *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(v[j].x, v[j].y, 0u, 0u);
+          for (int j = 0; j < PER; ++j) {
+            const int q = ct + j * 32 * kMx8ConvWarps;
+            const int r = q >> 3, c = q & 7;
+            *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(v[j].x, v[j].y, 0u, 0u);
+          }
+          fence_proxy_async_smem();   // the widened tile is read by the tensor core (async proxy)
         }
-        fence_proxy_async_smem();   // the widened tile is read by the tensor core (async proxy)
         __syncwarp();
         if (lane == 0) mbar_arrive(&conv[s]);
         if (++s == STAGES) { s = 0; ph ^= 1u; }

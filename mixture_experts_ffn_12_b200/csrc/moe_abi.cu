@@ -661,7 +661,7 @@ void moe_set_stage_events(void* const* starts, void* const* stops, int32_t n) {
 uint64_t moe_launch_count(void) { return moe::g_launches.load(); }
 
 moe_status_t moe_set_expert_gemm_variant(int32_t variant) {
-  if (variant < 0 || variant > 6) return MOE_ERR_INVALID_ARG;
+  if (variant < 0 || variant > 7) return MOE_ERR_INVALID_ARG;
   moe::g_gemm_variant.store(variant);
   return MOE_OK;
 }

@@ -110,3 +110,25 @@ def test_layer_a8_full_size_sampled(api):
     toks = np.unique(np.concatenate([[0, spec.T - 1], rng.choice(spec.T, 46, replace=False),
                                      sor[off[0]:off[1]][:16] // spec.k]))
     _check(api, spec, layer, toks)
+
+
+@pytest.mark.parametrize("spec", [MX8_SMALL, MX8_RAGGED, MX8_MANY, W.GPTOSS20B_MXFP4], ids=lambda s: s.name)
+def test_layer_a8_unpacked_weights_match_widened(api, spec):
+    """Whole 128-code K blocks of the E2M1 weights through TMA's 4-bit unpacking type (the
+    default) against every stage widened by the converter warps (expert-GEMM variant 7): the
+    same tiles reach the tensor core, so the outputs agree bit for bit.  K = 128 (all blocks
+    unpacked), 192 and 320 (a 64-code tail widened), 64 (no whole block) and 2880."""
+    layer = layer_for(spec)
+    d = api.upload_layer(layer)
+    ew = api.expert_weights_from(d)
+    cfg = api.config_from_spec(spec, y_f32=True, wfmt="mxfp4_a8")
+    outs = []
+    for variant in (0, 7):
+        api.set_expert_gemm_variant(variant)
+        try:
+            outs.append(api.layer_forward(cfg, d["x"], d["w_router"], d["b_router"], ew))
+            torch.cuda.synchronize()
+        finally:
+            api.set_expert_gemm_variant(0)
+        assert api.last_device_error() == 0
+    assert torch.equal(outs[0].view(torch.int32), outs[1].view(torch.int32))
