@@ -132,3 +132,30 @@ def test_layer_a8_unpacked_weights_match_widened(api, spec):
             api.set_expert_gemm_variant(0)
         assert api.last_device_error() == 0
     assert torch.equal(outs[0].view(torch.int32), outs[1].view(torch.int32))
+
+
+def test_layer_a8_weights_off_32_byte_alignment(api):
+    """E2M1 weights 16 bytes past a 32-byte boundary cannot be described to TMA's 4-bit
+    unpacking type (it wants 32-byte aligned bases): every stage is then widened by the
+    converter warps, and the output is the same bit for bit as with aligned weights."""
+    spec = MX8_RAGGED
+    layer = layer_for(spec)
+    d = api.upload_layer(layer)
+    ew = api.expert_weights_from(d)
+    cfg = api.config_from_spec(spec, y_f32=True, wfmt="mxfp4_a8")
+
+    def shifted(t):
+        buf = torch.empty(t.numel() + 16, dtype=t.dtype, device=t.device)
+        v = buf[16:].view(t.shape)
+        v.copy_(t)
+        assert v.data_ptr() % 32 == 16
+        return v
+
+    ew_off = api.ExpertWeights(shifted(ew.w_gate), shifted(ew.w_up), shifted(ew.w_down), ew.b_gate, ew.b_up,
+                               ew.b_down, ew.s_gate, ew.s_up, ew.s_down)
+    outs = []
+    for w in (ew, ew_off):
+        outs.append(api.layer_forward(cfg, d["x"], d["w_router"], d["b_router"], w))
+        torch.cuda.synchronize()
+        assert api.last_device_error() == 0
+    assert torch.equal(outs[0].view(torch.int32), outs[1].view(torch.int32))
