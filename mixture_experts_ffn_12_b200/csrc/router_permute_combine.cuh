@@ -469,14 +469,55 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(const int32_t* __res
   if (tid == blockDim.x - 1) expert_off[E] = warp_tot[(blockDim.x >> 5) - 1];
 }
 
+// Chunk c's first row per expert is base[e * nchunks + c] (from permute_scan_kernel), or,
+// with base == nullptr (few counts: E * nchunks <= kScatterScanMax), this CTA works it out
+// from the chunk counts itself -- the same exclusive scan over the expert-major (expert,
+// chunk) order -- and CTA 0 writes expert_off; one kernel boundary fewer in the dispatch.
+constexpr int kScatterScanMax = 4096;
+
 __global__ void __launch_bounds__(kChunk) permute_scatter_kernel(const int32_t* __restrict__ ids, int T, int k, int E,
                                                                  int nchunks, const int32_t* __restrict__ base,
+                                                                 const int32_t* __restrict__ chunk_cnt,
+                                                                 int32_t* __restrict__ expert_off,
                                                                  int32_t* __restrict__ row_of_slot,
                                                                  int32_t* __restrict__ slot_of_row) {
   pdl_enter();
   __shared__ uint32_t mask[kChunkWarps][256];
-  build_masks(mask, ids, T, k, E);
+  __shared__ int base_s[256];
+  __shared__ int warp_tot[kChunkWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (base == nullptr) {
+    // thread e (< E <= 256): expert e's rows in all chunks and in the chunks before this one
+    int tot = 0, pre = 0;
+    if (static_cast<int>(threadIdx.x) < E) {
+      const int32_t* ce = chunk_cnt + static_cast<size_t>(threadIdx.x) * nchunks;
+      for (int c = 0; c < nchunks; ++c) {
+        const int v = ce[c];
+        tot += v;
+        pre += c < static_cast<int>(blockIdx.x) ? v : 0;
+      }
+    }
+    int incl = tot;   // exclusive scan of the totals over the experts
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += o;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    const int ex = before + incl - tot;
+    if (static_cast<int>(threadIdx.x) < E) {
+      base_s[threadIdx.x] = ex + pre;
+      if (blockIdx.x == 0) {
+        expert_off[threadIdx.x] = ex;
+        if (static_cast<int>(threadIdx.x) == E - 1) expert_off[E] = ex + tot;
+      }
+    }
+    __syncthreads();
+  }
+  build_masks(mask, ids, T, k, E);
   const int t = blockIdx.x * kChunk + threadIdx.x;
   if (t >= T) return;
   const uint32_t lt = (1u << lane) - 1u;
@@ -484,7 +525,8 @@ __global__ void __launch_bounds__(kChunk) permute_scatter_kernel(const int32_t* 
   for (int j = 0; j < k; ++j) {
     const int e = ids[static_cast<size_t>(t) * k + j];
     if (e < 0 || e >= E) continue;
-    int r = base[static_cast<size_t>(e) * nchunks + blockIdx.x] + __popc(mask[warp][e] & lt);
+    int r = (base != nullptr ? base[static_cast<size_t>(e) * nchunks + blockIdx.x] : base_s[e]) +
+            __popc(mask[warp][e] & lt);
     for (int w = 0; w < warp; ++w) r += __popc(mask[w][e]);
     if (r < 0 || r >= R) {
       flag_error(DEVERR_BOUNDS);
@@ -640,10 +682,15 @@ cudaError_t permute(const Launch& L, bool bf16, int64_t T, int D, int E, int k, 
     int32_t* cnt = scratch;
     int32_t* base = scratch + static_cast<size_t>(nchunks) * E;
     pdl_launch(permute_count_kernel, dim3(nchunks), dim3(kChunk), 0, L.stream, ids, static_cast<int>(T), k, E, nchunks, cnt);
-    pdl_launch(permute_scan_kernel, dim3(1), dim3(1024), 0, L.stream, cnt, nchunks * E, E, nchunks, base, expert_off);
-    pdl_launch(permute_scatter_kernel, dim3(nchunks), dim3(kChunk), 0, L.stream, ids, static_cast<int>(T), k, E, nchunks, base,
-                                                             row_of_slot, slot_of_row);
-    count_launch(3);
+    const bool scan_here = static_cast<int64_t>(E) * nchunks <= kScatterScanMax;
+    if (!scan_here) {
+      pdl_launch(permute_scan_kernel, dim3(1), dim3(1024), 0, L.stream, cnt, nchunks * E, E, nchunks, base, expert_off);
+      count_launch();
+    }
+    pdl_launch(permute_scatter_kernel, dim3(nchunks), dim3(kChunk), 0, L.stream, ids, static_cast<int>(T), k, E, nchunks,
+               scan_here ? static_cast<const int32_t*>(nullptr) : static_cast<const int32_t*>(base),
+               static_cast<const int32_t*>(cnt), expert_off, row_of_slot, slot_of_row);
+    count_launch(2);
   }
   if (x != nullptr && x_perm != nullptr) {
     const int R = static_cast<int>(T * k);
