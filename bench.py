@@ -296,8 +296,10 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through MoELayer.run_host_batches: every step copies its input from
     # pinned host memory and its output back to pinned host memory; the copies of
-    # neighbouring steps overlap the forward (three streams, double-buffered)
-    Ke = max(5, K // 4)
+    # neighbouring steps overlap the forward (three streams, double-buffered).  The same
+    # K steps as the device-timed region: the first step's copy in and the last step's
+    # copy out (~0.5 ms each at the prefill shape) do not overlap a forward
+    Ke = K
     xs_host = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for _ in range(2)]
     for xh in xs_host:
         xh.copy_(x)
