@@ -450,10 +450,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sb = sa + LY::A_BYTES;
           const int half = hsplit ? kb / KB : 0;
           const int kbl = kb - half * KB;
-          if (hsplit) tma_load_3d(sa, &tmA, &full[s], kbl * BK, half, ti.m0);
-          else tma_load_2d(sa, &tmA, &full[s], kb * BK, ti.m0);
+          // the weight boxes first: they come more often from HBM or the other die than the
+          // activation rows, which neighbouring tiles reuse from L2
           tma_load_3d(sb, &tmB0, &full[s], kbl * BK, b_row, ti.g);
           if (NB == 2) tma_load_3d(sb + TN * kRowBytes, &tmB1, &full[s], kb * BK, ti.n0, ti.g);
+          if (hsplit) tma_load_3d(sa, &tmA, &full[s], kbl * BK, half, ti.m0);
+          else tma_load_2d(sa, &tmA, &full[s], kb * BK, ti.m0);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
